@@ -1,0 +1,393 @@
+#!/usr/bin/env python3
+"""Benchmark: sparse prefill attention layer (selection + sparse attention) on B200.
+
+One step = one pass of the whole hot path over one attention layer of the
+Llama-3.1-8B shape at L = 131072 (B = 1, 32 q heads, 8 kv heads, d = 128,
+causal, bf16): ``sparse_prefill_plan`` (anchor selection, theta = 5, sink 128,
+local 256) followed by ``sparse_prefill_attn``.  Inputs come from the seeded
+synthetic generator of ``workloads`` (sink bias + planted needles) and are
+resident in HBM before the timed region; at 1.5 GB they are larger than L2.
+
+Metric: kept-FLOP throughput (4 * d * sum_i |K_i| per layer) in TFLOP/s over
+the whole step; ``ms_per_step`` is ms per layer.  Extra keys: the attention
+kernel's roofline fraction, the SALE mode and the same kernel run dense, an
+end-to-end number through host buffers, clocks sampled during the timed
+region, and the CPU oracle timed on a bounded sample.
+
+Multi-GPU (``torchrun --nproc-per-node N``): every rank processes its own
+layer (independent problems, weak scaling, no collective on the data path);
+the timed region is bracketed by barriers and the max over ranks is reported.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from workloads import C2_LLAMA_128K, CONFIGS, Workload, generate  # noqa: E402
+
+METRIC = "sparse prefill attn ms/layer @128K & kept-FLOP TFLOP/s vs bf16 peak"
+UNIT = "TFLOP/s (kept FLOPs, plan+attn)"
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return dict(hbm=float(d["hbm_gbs"]), bf16=float(d["bf16_tflops"]),
+                    bf16_sus=float(d["bf16_tflops_sustained"]), src="measured")
+    except Exception:
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is None:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def _dist():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def oracle_sample(w: Workload, inp, theta: float, n_blocks: int = 3):
+    """CPU oracle on a bounded sample: anchor selection + sparse attention for the
+    last ``n_blocks`` query blocks of q head 0 (every row of those blocks)."""
+    from oracle import attention as oatt
+    from oracle import selection as osel
+    from workloads import bf16_bits_to_f32
+    qh = bf16_bits_to_f32(inp.q[0, 0]).astype(np.float64)
+    kh = bf16_bits_to_f32(inp.k[0, 0]).astype(np.float64)
+    vh = bf16_bits_to_f32(inp.v[0, 0]).astype(np.float64)
+    L = w.seq_len
+    nqb = (L + 127) // 128
+    blocks = list(range(nqb - n_blocks, nqb))
+    t0 = time.perf_counter()
+    sel = {qb: osel.anchor_block(qh, kh, qb, bq=128, sink=w.sink, local=w.local,
+                                 theta=theta).kept for qb in blocks}
+    rows = range(blocks[0] * 128, L)
+    oatt.attend_rows(qh, kh, vh, rows, lambda i: i // 128, lambda b: sel[b], bq=128,
+                     sink=w.sink, local=w.local)
+    dt = time.perf_counter() - t0
+    pairs = sum(oatt.kept_pairs_block(qb, L, bq=128, sink=w.sink, local=w.local,
+                                      n_selected=len(sel[qb])) for qb in blocks)
+    flops = 4 * 128 * pairs
+    cores = len(os.sched_getaffinity(0))
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max((i.get("num_threads", 1) for i in info), default=cores)
+    except Exception:
+        pass
+    return dict(value=flops / dt / 1e12, unit=UNIT, cores=cores, kind="oracle",
+                sample=f"q head 0, last {n_blocks} query blocks ({len(rows)} rows) of "
+                       f"{w.name}: anchor selection + fp64 sparse attention; {dt:.1f} s",
+                seconds=dt, flops=flops)
+
+
+def run_reference(args, w: Workload):
+    world, rank, _ = _dist()
+    if rank != 0:
+        return
+    inp = generate(w, kv_groups=[0])
+    vals = []
+    for _ in range(args.warmup_ref):
+        oracle_sample(w, inp, args.theta, n_blocks=1)
+    for _ in range(args.steps):
+        vals.append(oracle_sample(w, inp, args.theta, n_blocks=1))
+    v = statistics.median(x["value"] for x in vals)
+    cb = dict(vals[-1])
+    cb["value"] = v
+    for key in ("seconds", "flops"):
+        cb.pop(key, None)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": _config(w, args),
+            "cpu_baseline": cb, "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
+                                        "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def _config(w: Workload, args):
+    return {"workload": w.name, "batch": w.batch, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
+            "seq_len": w.seq_len, "head_dim": 128, "causal": True, "mode": args.mode,
+            "theta": args.theta, "sink": w.sink, "local": w.local, "block_q": 128,
+            "l2": "inputs (1.5 GB) larger than L2; no flush",
+            "parallelism": "independent layer per GPU"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--mode", default="anchor", choices=["anchor", "sale", "dense"])
+    ap.add_argument("--theta", type=float, default=5.0)
+    ap.add_argument("--config", default=C2_LLAMA_128K.name, choices=sorted(CONFIGS))
+    ap.add_argument("--no-extras", action="store_true", help="skip SALE/dense/e2e/cpu legs")
+    ap.add_argument("--warmup-ref", type=int, default=0)
+    args = ap.parse_args()
+    w = CONFIGS[args.config]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import block_sparse_long_sm_b200 as spa
+
+    world, rank, local = _dist()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    inp = generate(w)
+    q_h = torch.from_numpy(inp.q.view(np.int16)).view(torch.bfloat16).pin_memory()
+    k_h = torch.from_numpy(inp.k.view(np.int16)).view(torch.bfloat16).pin_memory()
+    v_h = torch.from_numpy(inp.v.view(np.int16)).view(torch.bfloat16).pin_memory()
+    q = q_h.to(dev)
+    k = k_h.to(dev)
+    v = v_h.to(dev)
+    B, Hq, Hkv, L = w.batch, w.heads_q, w.heads_kv, w.seq_len
+    o = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
+    p = spa.make_params(B, Hq, Hkv, L, mode=args.mode, sink=w.sink, local=w.local,
+                        theta=args.theta, tau=w.tau, block_k=w.block_k if args.mode == "sale" else None)
+    ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
+
+    def step():
+        spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream), "plan")
+        spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None, stream=stream), "attn")
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    st, stats = spa.sparse_prefill_stats(p, ws, stream=stream)
+    spa.check(st, "stats")
+    flops_step = spa.kept_flops(stats)
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream), "plan")
+            ev[i][1].record(stream)
+            spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None, stream=stream), "attn")
+            ev[i][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    plan_ms = [a.elapsed_time(b) for a, b, _ in ev]
+    attn_ms = [b.elapsed_time(c) for _, b, c in ev]
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_step = total_ms / args.steps
+    value = flops_step * world * args.steps / (total_ms / 1e3) / 1e12
+    peaks = _peaks()
+    attn_avg = sum(attn_ms) / len(attn_ms)
+    achieved = flops_step / (attn_avg / 1e3) / 1e12
+    extras = {}
+    n_launch_plan = {"anchor": 3, "sale": 6, "dense": 0}[args.mode]
+    launches = (n_launch_plan + 1) * args.steps
+
+    if rank == 0 and not args.no_extras:
+        extras = bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, stats)
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": _config(w, args),
+            "plan_ms": statistics.median(plan_ms), "attn_ms": statistics.median(attn_ms),
+            "kept_fraction": stats.kept_pairs / stats.dense_pairs,
+            "kept_flops_per_layer": flops_step,
+            "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel",
+                         "achieved": achieved, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
+                         "frac": achieved / peaks["bf16_sus"], "traffic": None,
+                         "peak_source": f"{peaks['src']} bf16 dense, sustained (kernel timed inside a long loop)"},
+            "clocks": clk.summary(),
+            "gpu_launches": launches,
+        }
+        line.update(extras)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, stats):
+    """Selection roofline, SALE mode, dense mode, end-to-end and the CPU baseline."""
+    peaks = _peaks()
+    out = {}
+    B, Hq, Hkv, L = w.batch, w.heads_q, w.heads_kv, w.seq_len
+
+    def timed(fn, reps=3):
+        ts = []
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    # selection roofline (anchor plan): algorithmic bytes = read Q + read K once + write lists
+    p = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=w.sink, local=w.local, theta=args.theta)
+    ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
+    spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream))
+    st, s = spa.sparse_prefill_stats(p, ws, stream=stream)
+    plan_ms = timed(lambda: spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream)))
+    alg_bytes = 2 * B * Hq * L * 128 + 2 * B * Hkv * L * 128 + 4 * s.kept_candidates
+    gbs = alg_bytes / (plan_ms / 1e3) / 1e9
+    out["selection"] = {"mode": "anchor", "ms": plan_ms, "algorithmic_bytes": alg_bytes,
+                        "achieved_gbs": gbs, "peak_gbs": peaks["hbm"],
+                        "frac": gbs / peaks["hbm"], "kept_candidates": s.kept_candidates,
+                        "candidates": s.candidates}
+    del ws
+
+    # dense mode: same attention kernel over every causal key
+    pd = spa.make_params(B, Hq, Hkv, L, mode="dense", sink=w.sink, local=w.local)
+    wsd = torch.empty(spa.sparse_prefill_workspace_bytes(pd), dtype=torch.uint8, device=dev)
+    spa.check(spa.sparse_prefill_plan(pd, q, k, wsd, stream=stream))
+    dense_ms = timed(lambda: spa.check(spa.sparse_prefill_attn(pd, q, k, v, wsd, o, None, stream=stream)))
+    st, sd = spa.sparse_prefill_stats(pd, wsd, stream=stream)
+    dflops = spa.kept_flops(sd)
+    out["dense"] = {"attn_ms": dense_ms, "tflops": dflops / (dense_ms / 1e3) / 1e12,
+                    "frac": dflops / (dense_ms / 1e3) / 1e12 / peaks["bf16_sus"]}
+    del wsd
+
+    # SALE mode
+    ps = spa.make_params(B, Hq, Hkv, L, mode="sale", sink=w.sink, local=w.local, tau=w.tau,
+                         block_k=w.block_k)
+    wss = torch.empty(spa.sparse_prefill_workspace_bytes(ps), dtype=torch.uint8, device=dev)
+    spa.check(spa.sparse_prefill_plan(ps, q, k, wss, stream=stream))
+    sale_plan = timed(lambda: spa.check(spa.sparse_prefill_plan(ps, q, k, wss, stream=stream)))
+    sale_attn = timed(lambda: spa.check(spa.sparse_prefill_attn(ps, q, k, v, wss, o, None, stream=stream)))
+    st, ss = spa.sparse_prefill_stats(ps, wss, stream=stream)
+    sflops = spa.kept_flops(ss)
+    int_ops = 2 * 128 * (ss.candidates * 128)    # scan: every candidate (row, key) pair, per block row
+    out["sale"] = {"tau": w.tau, "block_k": w.block_k, "plan_ms": sale_plan, "attn_ms": sale_attn,
+                   "kept_fraction": ss.kept_pairs / ss.dense_pairs,
+                   "kept_tflops": sflops / ((sale_plan + sale_attn) / 1e3) / 1e12}
+    del wss
+
+    # end to end through host buffers: H2D of Q/K/V, plan + attn, D2H of O
+    o_h = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
+    pe = spa.make_params(B, Hq, Hkv, L, mode=args.mode, sink=w.sink, local=w.local,
+                         theta=args.theta, tau=w.tau,
+                         block_k=w.block_k if args.mode == "sale" else None)
+    wse = torch.empty(spa.sparse_prefill_workspace_bytes(pe), dtype=torch.uint8, device=dev)
+
+    def e2e():
+        q.copy_(q_h, non_blocking=True)
+        k.copy_(k_h, non_blocking=True)
+        v.copy_(v_h, non_blocking=True)
+        spa.check(spa.sparse_prefill_plan(pe, q, k, wse, stream=stream))
+        spa.check(spa.sparse_prefill_attn(pe, q, k, v, wse, o, None, stream=stream))
+        o_h.copy_(o, non_blocking=True)
+    e2e()
+    e_ms = timed(e2e, reps=3)
+    st, se = spa.sparse_prefill_stats(pe, wse, stream=stream)
+    out["e2e"] = {"value": spa.kept_flops(se) / (e_ms / 1e3) / 1e12, "unit": UNIT,
+                  "ms_per_step": e_ms,
+                  "h2d_bytes_per_step": 2 * (q.numel() + k.numel() + v.numel()),
+                  "d2h_bytes_per_step": 2 * o.numel()}
+    del wse
+
+    # CPU oracle on a bounded sample (same metric and unit)
+    if int(os.environ.get("WORLD_SIZE", "1")) == 1:
+        inp = generate(w, kv_groups=[0])
+        cb = oracle_sample(w, inp, args.theta, n_blocks=2)
+        cb.pop("seconds", None)
+        cb.pop("flops", None)
+        out["cpu_baseline"] = cb
+    return out
+
+
+if __name__ == "__main__":
+    main()

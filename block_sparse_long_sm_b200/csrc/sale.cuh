@@ -1,0 +1,344 @@
+// sale.cuh -- SALE-mode key-block selection (SALE: Low-bit Estimation for
+// Efficient Sparse Attention in Long-context LLM Prefilling, Sec. 3.2-3.4).
+//
+//   kmean_partial_kernel / kmean_final_kernel
+//       per (b, kv head): mean of K over the sequence, summed in fp64 over
+//       fixed chunks and rounded once to fp32 (smoothing, as SageAttention2).
+//   quant_kernel
+//       symmetric per-block 4-bit codes held in int8: scale = absmax / 7 and
+//       code = round-half-even(x / scale) in IEEE fp32, clamped to [-7, 7];
+//       K is smoothed first; an all-zero block gets scale 1.
+//   sale_scan_kernel
+//       per query block on the int8 tensor cores (tcgen05 kind::i8, M = 128,
+//       N = 256): first the sink-local tiles give em_i, el_i and the row
+//       threshold t_i = em_i + ln(tau * el_i) (Eq. (4) as corrected); then
+//       every candidate tile: a key block is kept when some valid row's
+//       largest estimated score in it reaches t_i.  The integer dot products
+//       are compared through max(dot) * (s_q * s_k * scale) >= t_i, exact in
+//       the integer part.  Output: one bit per key block.
+#pragma once
+
+#include "attn.cuh"
+#include "ptx.cuh"
+
+namespace spa {
+
+constexpr int kKmeanChunks = 64;
+
+struct KmeanArgs {
+  const __nv_bfloat16* k;   // [B*Hkv][L][128]
+  int L;
+  double* partial;          // [B*Hkv][chunks][128]
+  float* mean;              // [B*Hkv][128]
+};
+
+__global__ void kmean_partial_kernel(const KmeanArgs a) {
+  const int bkv = blockIdx.y, chunk = blockIdx.x, d = threadIdx.x;
+  const int per = (a.L + kKmeanChunks - 1) / kKmeanChunks;
+  const int r0 = chunk * per, r1 = min(r0 + per, a.L);
+  const __nv_bfloat16* kp = a.k + (long long)bkv * a.L * 128 + d;
+  double s = 0.0;
+  for (int r = r0; r < r1; ++r) s += static_cast<double>(__bfloat162float(kp[(long long)r * 128]));
+  a.partial[((long long)bkv * kKmeanChunks + chunk) * 128 + d] = s;
+}
+
+__global__ void kmean_final_kernel(const KmeanArgs a) {
+  const int bkv = blockIdx.x, d = threadIdx.x;
+  double s = 0.0;
+  for (int c = 0; c < kKmeanChunks; ++c) s += a.partial[((long long)bkv * kKmeanChunks + c) * 128 + d];
+  a.mean[(long long)bkv * 128 + d] = static_cast<float>(s / static_cast<double>(a.L));
+}
+
+struct QuantArgs {
+  const __nv_bfloat16* x;   // [heads][L][128]
+  const float* mean;        // [heads][128] or null (no smoothing)
+  int L, rows;              // rows per quantisation block
+  int nblk;                 // blocks per head
+  int8_t* codes;            // [heads][L][128]
+  float* scales;            // [heads][nblk]
+};
+
+// grid (nblk, heads), 128 threads: thread d owns column d of the block.
+__global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
+  const int head = blockIdx.y, blk = blockIdx.x, d = threadIdx.x;
+  const int r0 = blk * a.rows, r1 = min(r0 + a.rows, a.L);
+  const __nv_bfloat16* xp = a.x + (long long)head * a.L * 128 + d;
+  const float mu = a.mean ? a.mean[(long long)head * 128 + d] : 0.f;
+  float amax = 0.f;
+  for (int r = r0; r < r1; ++r) {
+    const float v = __fsub_rn(__bfloat162float(xp[(long long)r * 128]), mu);
+    amax = fmaxf(amax, fabsf(v));
+  }
+  __shared__ float red[4];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  if ((d & 31) == 0) red[d >> 5] = amax;
+  __syncthreads();
+  amax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const float sc = amax > 0.f ? __fdiv_rn(amax, 7.0f) : 1.0f;
+  int8_t* cp = a.codes + (long long)head * a.L * 128 + d;
+  for (int r = r0; r < r1; ++r) {
+    const float v = __fsub_rn(__bfloat162float(xp[(long long)r * 128]), mu);
+    float c = rintf(__fdiv_rn(v, sc));
+    c = fminf(fmaxf(c, -7.f), 7.f);
+    cp[(long long)r * 128] = static_cast<int8_t>(c);
+  }
+  if (d == 0) a.scales[(long long)head * a.nblk + blk] = sc;
+}
+
+// ---------------------------------------------------------------------------
+// fused sink-local statistics + block scan
+// ---------------------------------------------------------------------------
+constexpr int kSaleThreads = 320;            // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
+constexpr int kSaleStages = 3;
+constexpr uint32_t kQ8Bytes = 128u * 128u;   // 128 rows x 128 int8
+constexpr uint32_t kK8Bytes = 256u * 128u;   // 256 rows x 128 int8
+constexpr int kMaxGroupWords = 512;          // candidate 16-key groups / 32 (L <= 262144)
+constexpr uint32_t kSaleSmemBytes =
+    1024u + kQ8Bytes + kSaleStages * kK8Bytes + 512u + kMaxGroupWords * 4u + 128u * 16u;
+
+struct SaleArgs {
+  int B, Hq, Hkv, L, nqb, group;
+  int sink, local, bk, nkb;
+  float scale, tau;
+  const float* sq;          // [B*Hq][nqb]
+  const float* sk;          // [B*Hkv][nkb]
+  uint32_t* mask;           // [B*Hq*nqb][nwords] over key blocks
+  int nwords;
+  uint32_t* err;
+  uint64_t wait_ns;
+};
+
+__global__ void __launch_bounds__(kSaleThreads, 1)
+sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
+                 const __grid_constant__ CUtensorMap tm_k8, const SaleArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_q = s_base;
+  auto s_k = [&](int st) { return s_base + kQ8Bytes + st * kK8Bytes; };
+  uint8_t* bar_area = smem + kQ8Bytes + kSaleStages * kK8Bytes;
+  const uint32_t b0 = smem_u32(bar_area);
+  const uint32_t bar_q = b0;
+  auto bar_full = [&](int s) { return b0 + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return b0 + 8u * (1 + kSaleStages + s); };
+  const uint32_t bar_sfull0 = b0 + 8u * (1 + 2 * kSaleStages);
+  const uint32_t bar_sfree0 = bar_sfull0 + 16u;
+  const uint32_t bar_drain = bar_sfull0 + 32u;
+  const uint32_t bar_stat = bar_sfull0 + 40u;     // both column halves of every row posted
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 8 * (1 + 2 * kSaleStages) + 48);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+  uint32_t* gflags = reinterpret_cast<uint32_t*>(bar_area + 512);       // candidate group flags
+  float* part = reinterpret_cast<float*>(gflags + kMaxGroupWords);      // [128][4]: m,l of 2 halves
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int x = blockIdx.x;
+  const int bh = x / a.nqb, qb = x - (x / a.nqb) * a.nqb;
+  const int b = bh / a.Hq, h = bh - b * a.Hq;
+  const int bkv = b * a.Hkv + h / a.group;
+  const int row0 = qb * 128;
+  const int le = min(row0 + 128, a.L);
+  const int ls = max(0, row0 + 128 - a.local);
+  const int sink_end = min(a.sink, ls);
+  // tiles of 256 keys: sink, local (statistics), then candidates (scan)
+  const int n_sink_t = (sink_end + 255) / 256;
+  const int n_loc_t = (le - ls + 255) / 256;
+  const int cand_lo = a.sink, cand_hi = max(a.sink, ls);
+  const int n_cand_t = (cand_hi - cand_lo + 255) / 256;
+  const int n_stat_t = n_sink_t + n_loc_t;
+  const int T = n_stat_t + n_cand_t;
+  const int n_groups = (cand_hi - cand_lo) / 16;
+  auto tile_key0 = [&](int t) {
+    if (t < n_sink_t) return t * 256;
+    if (t < n_stat_t) return ls + (t - n_sink_t) * 256;
+    return cand_lo + (t - n_stat_t) * 256;
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < kSaleStages; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_sfull0 + 8u * i, 1);
+      mbar_init(bar_sfree0 + 8u * i, 256);
+    }
+    mbar_init(bar_drain, 1);
+    mbar_init(bar_stat, 256);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  for (int i = threadIdx.x; i < kMaxGroupWords; i += blockDim.x) gflags[i] = 0u;
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtx wc{abort_flag, a.err, a.wait_ns};
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, kQ8Bytes);
+      tma_load_2d(s_q, &tm_q8, bar_q, 0, bh * a.L + row0);
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t % kSaleStages;
+        if (t >= kSaleStages && !mbar_wait(bar_empty(st), ((t / kSaleStages) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(bar_full(st), kK8Bytes);
+        tma_load_2d(s_k(st), &tm_k8, bar_full(st), 0, bkv * a.L + tile_key0(t));
+        issued = t + 1;
+      }
+      {  // no copy may still be in flight when the CTA exits
+        mbar_drain(bar_q, 0, a.wait_ns);
+        for (int t = max(0, issued - kSaleStages); t < issued; ++t)
+          mbar_drain(bar_full(t % kSaleStages), (t / kSaleStages) & 1, a.wait_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(bar_q, 0, wc);
+      for (int t = 0; ok && t < T; ++t) {
+        const int st = t % kSaleStages, bb = t & 1;
+        if (!(ok = mbar_wait(bar_full(st), (t / kSaleStages) & 1, wc))) break;
+        if (t >= 2 && !(ok = mbar_wait(bar_sfree0 + 8u * bb, ((t - 2) >> 1) & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+          mma_i8_ss(tmem + 256u * bb, smem_desc_sw128(s_q + ks * 32u, 16),
+                    smem_desc_sw128(s_k(st) + ks * 32u, 16), kIdescI8, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_sfull0 + 8u * bb);
+        mma_commit(bar_empty(st));
+      }
+      mma_commit(bar_drain);
+      mbar_drain(bar_drain, 0, a.wait_ns);
+    }
+    __syncwarp();
+  } else {
+    const int ew = warp - 2;                 // 0..7
+    const int quad = warp & 3;               // TMEM lane quadrant
+    const int half = ew >> 2;                // columns [128*half, 128*half + 128)
+    const int r = quad * 32 + lane;
+    const int row = row0 + r;
+    const bool row_valid = row < a.L;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const float cq = a.sq[(long long)bh * a.nqb + qb] * a.scale;
+    const float* skp = a.sk + (long long)bkv * a.nkb;
+    float m = -INFINITY, l = 0.f, thr = INFINITY;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int bb = t & 1;
+      if (!(ok = warp_wait(bar_sfull0 + 8u * bb, (t >> 1) & 1, wc))) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(tmem + lane_off + 256u * bb + 128u * half + 32u * c, sr[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar_sfree0 + 8u * bb);
+      const int key0 = tile_key0(t) + 128 * half;
+      if (t < n_stat_t) {
+        // S~ over the causal sink-local keys of this row
+        int limit;
+        if (t < n_sink_t) limit = sink_end - key0;
+        else limit = min(le - key0, row - key0 + 1);
+        limit = max(0, min(limit, 128));
+        float tm = -INFINITY;
+        float sv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const int col = c * 32 + e;
+            const int key = key0 + col;
+            const float sk = skp[min(key, a.L - 1) / a.bk];
+            const float v = col < limit
+                                ? static_cast<float>(static_cast<int>(sr[c][e])) * (cq * sk)
+                                : -INFINITY;
+            sv[c][e] = v;
+            tm = fmaxf(tm, v);
+          }
+        }
+        if (tm > -INFINITY) {
+          const float mn = fmaxf(m, tm);
+          float acc = 0.f;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e) acc += expf(sv[c][e] - mn);
+          l = l * expf(m - mn) + acc;
+          m = mn;
+        }
+        if (t == n_stat_t - 1) {
+          // merge the two column halves of each row, then t_i = em + ln(tau el)
+          part[r * 4 + half * 2 + 0] = m;
+          part[r * 4 + half * 2 + 1] = l;
+          mbar_arrive(bar_stat);
+          if (!(ok = warp_wait(bar_stat, 0, wc))) break;
+          const float m0 = part[r * 4 + 0], l0 = part[r * 4 + 1];
+          const float m1 = part[r * 4 + 2], l1 = part[r * 4 + 3];
+          const float em = fmaxf(m0, m1);
+          const float el = (m0 > -INFINITY ? l0 * expf(m0 - em) : 0.f) +
+                           (m1 > -INFINITY ? l1 * expf(m1 - em) : 0.f);
+          thr = row_valid ? em + logf(a.tau * el) : INFINITY;
+        }
+      } else {
+        // candidate tile: one flag per 16-key group (groups never straddle ls)
+        uint32_t gbits = 0;
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const int key = key0 + 16 * g;
+          int mx = INT_MIN;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = (16 * g + e) >> 5, ee = (16 * g + e) & 31;
+            mx = max(mx, static_cast<int>(sr[c][ee]));
+          }
+          if (key < cand_hi) {
+            const float sk = skp[key / a.bk];
+            if (static_cast<float>(mx) * (cq * sk) >= thr) gbits |= 1u << g;
+          }
+        }
+        gbits = __reduce_or_sync(0xffffffffu, gbits);
+        if (lane == 0 && gbits) {
+          const int g0 = (key0 - cand_lo) / 16;     // first group of this half-tile
+#pragma unroll
+          for (int g = 0; g < 8; ++g)
+            if ((gbits >> g) & 1u) atomicOr(&gflags[(g0 + g) >> 5], 1u << ((g0 + g) & 31));
+        }
+      }
+    }
+    (void)n_groups;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // key-block flags -> global bitmask row (every word of the row is written)
+  if (!*abort_flag) {
+    const int gpb = a.bk / 16;                     // groups per key block
+    const int kb_lo = cand_lo / a.bk;
+    uint32_t* mrow = a.mask + (long long)x * a.nwords;
+    for (int w = threadIdx.x; w < a.nwords; w += blockDim.x) {
+      uint32_t word = 0;
+      for (int bit = 0; bit < 32; ++bit) {
+        const int kb = w * 32 + bit;
+        if (kb < kb_lo || kb * a.bk >= cand_hi) continue;
+        const int g0 = (kb - kb_lo) * gpb;
+        bool any = false;
+        for (int g = g0; g < g0 + gpb; ++g) any |= (gflags[g >> 5] >> (g & 31)) & 1u;
+        word |= (any ? 1u : 0u) << bit;
+      }
+      mrow[w] = word;
+    }
+  }
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace spa

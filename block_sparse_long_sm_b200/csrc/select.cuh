@@ -1,0 +1,508 @@
+// select.cuh -- anchor-mode key selection (AnchorAttention: Difference-Aware
+// Sparse Attention with Stripe Granularity, Eq. (1)-(3)) and the generic
+// bitmask -> ascending-index-list compaction shared with SALE mode.
+//
+//   anchor_pool_kernel   per query block: S = Q [K_sink; K_local]^T on the
+//                        tensor cores, row max over the causal sink-local
+//                        keys (Eq. (1), the row-max buffer M), its mean over
+//                        the block (avgpool(x_a)), and the pooled query
+//                        avgpool(Q) * scale split into bf16 hi + lo parts.
+//   stripe_scan_kernel   per (128 query blocks) x (16 key tiles): the pooled
+//                        scores avgpool(Q) K^T * scale as one tcgen05 GEMM
+//                        (hi and lo products accumulated in fp32), the
+//                        difference-aware test of Eq. (2) and the candidate
+//                        range check, written as a key bitmask per block.
+//   compact_kernel       per query block: the bitmask's set bits in
+//                        ascending order, written with coalesced warp stores
+//                        into the block's list (Eq. (3): discrete key
+//                        coordinates), plus the count.
+#pragma once
+
+#include "attn.cuh"
+#include "ptx.cuh"
+
+namespace spa {
+
+// ---------------------------------------------------------------------------
+// anchor + pooling
+// ---------------------------------------------------------------------------
+constexpr int kPoolThreads = 192;
+constexpr int kPoolStages = 2;
+constexpr uint32_t kPoolSmemBytes = 1024u + kTileBytes + kPoolStages * kTileBytes + 256u;
+
+struct PoolArgs {
+  int B, Hq, Hkv, L, nqb, group;
+  int sink, local;
+  float scale;                  // softmax scale
+  float* xbar;                  // [B*Hq*nqb]
+  __nv_bfloat16* qbar;          // [2][B*Hq][nqb][128]: hi then lo
+  uint32_t* err;
+  uint64_t wait_ns;
+};
+
+__global__ void __launch_bounds__(kPoolThreads, 1)
+anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
+                   const __grid_constant__ CUtensorMap tm_k, const PoolArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_q = s_base;
+  auto s_k = [&](int st) { return s_base + kTileBytes + st * kTileBytes; };
+  uint8_t* bar_area = smem + kTileBytes + kPoolStages * kTileBytes;
+  const uint32_t b0 = smem_u32(bar_area);
+  const uint32_t bar_q = b0;
+  auto bar_full = [&](int s) { return b0 + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return b0 + 8u * (1 + kPoolStages + s); };
+  const uint32_t bar_sfull0 = b0 + 8u * (1 + 2 * kPoolStages);
+  const uint32_t bar_sfree0 = bar_sfull0 + 16u;
+  const uint32_t bar_drain = bar_sfull0 + 32u;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 8 * (1 + 2 * kPoolStages) + 40);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+  float* red = reinterpret_cast<float*>(tmem_holder + 2);   // 4 partial sums
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_q, 1);
+    for (int s = 0; s < kPoolStages; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_sfull0 + 8u * i, 1);
+      mbar_init(bar_sfree0 + 8u * i, 128);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtx wc{abort_flag, a.err, a.wait_ns};
+
+  // block geometry
+  const int x = blockIdx.x;
+  const int bh = x / a.nqb, qb = x - (x / a.nqb) * a.nqb;
+  const int b = bh / a.Hq, h = bh - b * a.Hq;
+  const int kvh = h / a.group;
+  const int row0 = qb * 128;
+  const int le = min(row0 + 128, a.L);
+  const int nrows = le - row0;
+  const int ls = max(0, row0 + 128 - a.local);
+  const int sink_end = min(a.sink, ls);
+  const int n_sink_t = (sink_end + 127) / 128;
+  const int n_loc_t = (le - ls + 127) / 128;
+  const int T = n_sink_t + n_loc_t;
+  const int kv_row0 = (b * a.Hkv + kvh) * a.L;
+  auto tile_key0 = [&](int t) { return t < n_sink_t ? t * 128 : ls + (t - n_sink_t) * 128; };
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_q, kTileBytes);
+      const int qrow = bh * a.L + row0;
+      tma_load_2d(s_q, &tm_q, bar_q, 0, qrow);
+      tma_load_2d(s_q + kHalfBytes, &tm_q, bar_q, 64, qrow);
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t % kPoolStages;
+        if (t >= kPoolStages && !mbar_wait(bar_empty(st), ((t / kPoolStages) - 1) & 1, wc)) break;
+        mbar_arrive_expect_tx(bar_full(st), kTileBytes);
+        tma_load_2d(s_k(st), &tm_k, bar_full(st), 0, kv_row0 + tile_key0(t));
+        tma_load_2d(s_k(st) + kHalfBytes, &tm_k, bar_full(st), 64, kv_row0 + tile_key0(t));
+        issued = t + 1;
+      }
+      {  // no copy may still be in flight when the CTA exits
+        mbar_drain(bar_q, 0, a.wait_ns);
+        for (int t = max(0, issued - kPoolStages); t < issued; ++t)
+          mbar_drain(bar_full(t % kPoolStages), (t / kPoolStages) & 1, a.wait_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(bar_q, 0, wc);
+      for (int t = 0; ok && t < T; ++t) {
+        const int st = t % kPoolStages, bb = t & 1;
+        if (!(ok = mbar_wait(bar_full(st), (t / kPoolStages) & 1, wc))) break;
+        if (t >= 2 && !(ok = mbar_wait(bar_sfree0 + 8u * bb, ((t - 2) >> 1) & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32u;
+          mma_bf16_ss(tmem + 128u * bb, smem_desc_sw128(s_q + off, 16),
+                      smem_desc_sw128(s_k(st) + off, 16), kIdescQK, ks > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_sfull0 + 8u * bb);
+        mma_commit(bar_empty(st));
+      }
+      mma_commit(bar_drain);
+      mbar_drain(bar_drain, 0, a.wait_ns);
+    }
+    __syncwarp();
+  } else {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    float mx = -INFINITY;
+    bool ok = true;
+    for (int t = 0; t < T; ++t) {
+      const int bb = t & 1;
+      if (!(ok = warp_wait(bar_sfull0 + 8u * bb, (t >> 1) & 1, wc))) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + 128u * bb + 32u * c, sr[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar_sfree0 + 8u * bb);
+      const int key0 = tile_key0(t);
+      // valid keys: sink tiles below sink_end; local tiles causal (j <= i) and below L
+      int limit = (t < n_sink_t) ? (sink_end - key0) : min(le - key0, row0 + r - key0 + 1);
+      limit = min(limit, 128);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (c * 32 + e < limit) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+    }
+    if (ok) {
+      const bool valid = r < nrows;
+      float xa = valid ? mx * a.scale : 0.f;
+      float s = xa;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (lane == 0) red[quad] = s;
+    }
+    // pooled query: thread r owns column d = r (Q is read from shared memory,
+    // so wait on its barrier as well)
+    if (ok) ok = warp_wait(bar_q, 0, wc);
+    if (ok) {
+      float acc = 0.f;
+      const int d = r;
+      const uint32_t half = (d >> 6) * kHalfBytes;
+      const uint32_t byte = (d & 63) * 2;
+      for (int rr = 0; rr < nrows; ++rr) {
+        const __nv_bfloat16 v =
+            *reinterpret_cast<const __nv_bfloat16*>(smem + half + sw128_offset(rr, byte));
+        acc += __bfloat162float(v);
+      }
+      const float qbar = (acc / static_cast<float>(nrows)) * a.scale;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(qbar);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(qbar - __bfloat162float(hi));
+      const long long base = ((long long)bh * a.nqb + qb) * 128 + d;
+      const long long lo_off = (long long)a.B * a.Hq * a.nqb * 128;
+      a.qbar[base] = hi;
+      a.qbar[lo_off + base] = lo;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 64 && !*abort_flag) {
+    a.xbar[(long long)bh * a.nqb + qb] = (red[0] + red[1] + red[2] + red[3]) / static_cast<float>(nrows);
+  }
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// pooled-score scan: bitmask[bh][qb][word] over keys
+// ---------------------------------------------------------------------------
+constexpr int kScanThreads = 192;
+constexpr int kScanStages = 3;
+constexpr int kScanTilesPerChunk = 16;
+constexpr uint32_t kScanSmemBytes = 1024u + 2u * kTileBytes + kScanStages * kTileBytes + 256u;
+
+struct ScanArgs {
+  int B, Hq, Hkv, L, nqb, group;
+  int sink, local;
+  float theta;
+  const float* xbar;
+  uint32_t* mask;        // [B*Hq*nqb][nwords]
+  int nwords;            // words per block row (multiple of 4)
+  uint32_t* err;
+  uint64_t wait_ns;
+};
+
+__global__ void __launch_bounds__(kScanThreads, 1)
+stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
+                   const __grid_constant__ CUtensorMap tm_k, const ScanArgs a) {
+  const int bh = blockIdx.z;
+  const int mt = blockIdx.y;
+  const int chunk = blockIdx.x;
+  const int qb_lo = mt * 128;
+  const int qb_hi = min(qb_lo + 128, a.nqb);
+  const int key_end = max(0, qb_hi * 128 - a.local);      // ls of the last block
+  if (key_end <= a.sink) return;
+  const int kt0 = a.sink / 128;
+  const int kt_end = (key_end + 127) / 128;
+  const int t_lo = kt0 + chunk * kScanTilesPerChunk;
+  const int t_hi = min(t_lo + kScanTilesPerChunk, kt_end);
+  if (t_lo >= t_hi) return;
+  const int T = t_hi - t_lo;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_a = s_base;                            // hi tile, then lo tile
+  auto s_k = [&](int st) { return s_base + 2u * kTileBytes + st * kTileBytes; };
+  uint8_t* bar_area = smem + 2 * kTileBytes + kScanStages * kTileBytes;
+  const uint32_t b0 = smem_u32(bar_area);
+  const uint32_t bar_a = b0;
+  auto bar_full = [&](int s) { return b0 + 8u * (1 + s); };
+  auto bar_empty = [&](int s) { return b0 + 8u * (1 + kScanStages + s); };
+  const uint32_t bar_sfull0 = b0 + 8u * (1 + 2 * kScanStages);
+  const uint32_t bar_sfree0 = bar_sfull0 + 16u;
+  const uint32_t bar_drain = bar_sfull0 + 32u;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 8 * (1 + 2 * kScanStages) + 40);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(bar_a, 1);
+    for (int s = 0; s < kScanStages; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_sfull0 + 8u * i, 1);
+      mbar_init(bar_sfree0 + 8u * i, 128);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtx wc{abort_flag, a.err, a.wait_ns};
+  const int b = bh / a.Hq, h = bh - b * a.Hq;
+  const int kv_row0 = (b * a.Hkv + h / a.group) * a.L;
+  const int BH = a.B * a.Hq;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar_a, 2 * kTileBytes);
+      tma_load_3d(s_a, &tm_qbar, bar_a, 0, qb_lo, bh);
+      tma_load_3d(s_a + kHalfBytes, &tm_qbar, bar_a, 64, qb_lo, bh);
+      tma_load_3d(s_a + kTileBytes, &tm_qbar, bar_a, 0, qb_lo, BH + bh);
+      tma_load_3d(s_a + kTileBytes + kHalfBytes, &tm_qbar, bar_a, 64, qb_lo, BH + bh);
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t % kScanStages;
+        if (t >= kScanStages && !mbar_wait(bar_empty(st), ((t / kScanStages) - 1) & 1, wc)) break;
+        const int key0 = (t_lo + t) * 128;
+        mbar_arrive_expect_tx(bar_full(st), kTileBytes);
+        tma_load_2d(s_k(st), &tm_k, bar_full(st), 0, kv_row0 + key0);
+        tma_load_2d(s_k(st) + kHalfBytes, &tm_k, bar_full(st), 64, kv_row0 + key0);
+        issued = t + 1;
+      }
+      {  // no copy may still be in flight when the CTA exits
+        mbar_drain(bar_a, 0, a.wait_ns);
+        for (int t = max(0, issued - kScanStages); t < issued; ++t)
+          mbar_drain(bar_full(t % kScanStages), (t / kScanStages) & 1, a.wait_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(bar_a, 0, wc);
+      for (int t = 0; ok && t < T; ++t) {
+        const int st = t % kScanStages, bb = t & 1;
+        if (!(ok = mbar_wait(bar_full(st), (t / kScanStages) & 1, wc))) break;
+        if (t >= 2 && !(ok = mbar_wait(bar_sfree0 + 8u * bb, ((t - 2) >> 1) & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {       // hi, then lo
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32u;
+            mma_bf16_ss(tmem + 128u * bb, smem_desc_sw128(s_a + part * kTileBytes + off, 16),
+                        smem_desc_sw128(s_k(st) + off, 16), kIdescQK,
+                        (part > 0 || ks > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(bar_sfull0 + 8u * bb);
+        mma_commit(bar_empty(st));
+      }
+      mma_commit(bar_drain);
+      mbar_drain(bar_drain, 0, a.wait_ns);
+    }
+    __syncwarp();
+  } else {
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int qb = qb_lo + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    const bool row_valid = qb < a.nqb;
+    const float xb = row_valid ? a.xbar[(long long)bh * a.nqb + qb] : 0.f;
+    const int cand_hi = row_valid ? max(0, (qb + 1) * 128 - a.local) : 0;   // ls of this block
+    uint32_t* mrow = a.mask + ((long long)bh * a.nqb + (row_valid ? qb : 0)) * a.nwords;
+    for (int t = 0; t < T; ++t) {
+      const int bb = t & 1;
+      if (!warp_wait(bar_sfull0 + 8u * bb, (t >> 1) & 1, wc)) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + 128u * bb + 32u * c, sr[c]);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar_sfree0 + 8u * bb);
+      const int key0 = (t_lo + t) * 128;
+      // candidate keys of this row inside the tile: [lo, hi)
+      const int lo = max(a.sink - key0, 0);
+      const int hi = min(cand_hi - key0, 128);
+      uint4 wv;
+      uint32_t* w = &wv.x;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t bits = 0;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float s = __uint_as_float(sr[c][e]);
+          bits |= ((xb - s) <= a.theta ? 1u : 0u) << e;
+        }
+        // keep only the candidate columns [lo, hi) of this word
+        const int wlo = c * 32, whi = c * 32 + 32;
+        const int l0 = max(lo, wlo) - wlo, l1 = min(hi, whi) - wlo;
+        uint32_t range = 0;
+        if (l1 > l0) range = (l1 - l0 >= 32 ? 0xffffffffu : ((1u << (l1 - l0)) - 1u)) << l0;
+        w[c] = bits & range;
+      }
+      if (row_valid && key0 < cand_hi) {
+        *reinterpret_cast<uint4*>(mrow + key0 / 32) = wv;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 256);
+}
+
+// ---------------------------------------------------------------------------
+// bitmask -> ascending index list
+// ---------------------------------------------------------------------------
+constexpr int kCompactThreads = 256;
+
+struct CompactArgs {
+  int nrows_total;          // B*Hq*nqb
+  int nqb;
+  int L;
+  int sink, local;
+  int unit;                 // 1: bits are keys; bk: bits are key blocks
+  const uint32_t* mask;     // [rows][nwords]
+  int nwords;
+  int* lists;
+  long long list_per_head;  // list elements per (b, h)
+  long long cap_a;          // local + sink
+  int* counts;
+};
+
+__global__ void __launch_bounds__(kCompactThreads)
+compact_kernel(const CompactArgs a) {
+  const int row = blockIdx.x;
+  const int bh = row / a.nqb, qb = row - (row / a.nqb) * a.nqb;
+  const int ls = max(0, (qb + 1) * 128 - a.local);
+  const int bit_lo = a.sink / a.unit;
+  const int bit_hi = max(a.sink, ls) / a.unit;
+  const int w_lo = bit_lo / 32;
+  const int w_hi = bit_hi > bit_lo ? (bit_hi + 31) / 32 : w_lo;
+  const int n = w_hi - w_lo;
+  const uint32_t* m = a.mask + (long long)row * a.nwords;
+  int* out = a.lists + (long long)bh * a.list_per_head + cap_prefix(qb, 128, a.cap_a) / a.unit;
+
+  __shared__ int warp_cnt[kCompactThreads / 32];
+  __shared__ int warp_base[kCompactThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = kCompactThreads / 32;
+  const int seg = (((n + nw - 1) / nw) + 31) & ~31;      // words per warp, multiple of 32
+  const int s_lo = w_lo + warp * seg;
+  const int s_hi = min(s_lo + seg, w_hi);
+  int cnt = 0;
+  for (int w = s_lo + lane; w < s_hi; w += 32) cnt += __popc(m[w]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) warp_cnt[warp] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int i = 0; i < nw; ++i) {
+      warp_base[i] = run;
+      run += warp_cnt[i];
+    }
+    a.counts[row] = run;
+  }
+  __syncthreads();
+  int base = warp_base[warp];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int w0 = s_lo; w0 < s_hi; w0 += 32) {
+    const uint32_t word = (w0 + lane < s_hi) ? m[w0 + lane] : 0u;
+    const int pc = __popc(word);
+    int incl = pc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - pc;
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t wj = __shfl_sync(0xffffffffu, word, j);
+      if (wj == 0u) continue;                         // warp-uniform
+      const int oj = __shfl_sync(0xffffffffu, excl, j);
+      if ((wj >> lane) & 1u) out[base + oj + __popc(wj & lt)] = 32 * (w0 + j) + lane;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// stats: totals over all query blocks into the workspace header
+// ---------------------------------------------------------------------------
+struct StatsArgs {
+  int nrows_total, nqb, L, sink, local, mode, unit;
+  const int* counts;
+  unsigned long long* acc;   // [5]: blocks, candidates, kept, kept_pairs, dense_pairs
+};
+
+__global__ void stats_kernel(const StatsArgs a) {
+  const int row = blockIdx.x * blockDim.x + threadIdx.x;
+  unsigned long long v[5] = {0, 0, 0, 0, 0};
+  if (row < a.nrows_total) {
+    const int qb = row % a.nqb;
+    const long long row0 = (long long)qb * 128;
+    const long long le = min(row0 + 128, (long long)a.L);
+    const long long n = le - row0;
+    const long long ls = max(0LL, row0 + 128 - a.local);
+    const long long sink_end = min((long long)a.sink, ls);
+    const long long cand = max(0LL, ls - a.sink);
+    const long long kept = (a.mode == kModeDense) ? 0 : (long long)a.counts[row] * a.unit;
+    // sum_{i=row0}^{le-1} (i + 1 - ls) and sum (i + 1)
+    const long long sum_i1 = (le * (le + 1) - row0 * (row0 + 1)) / 2;
+    v[0] = 1;
+    v[1] = (a.mode == kModeDense) ? 0 : cand;
+    v[2] = kept;
+    v[3] = (a.mode == kModeDense) ? sum_i1 : n * (sink_end + kept) + sum_i1 - n * ls;
+    v[4] = sum_i1;
+  }
+#pragma unroll
+  for (int k = 0; k < 5; ++k) {
+    unsigned long long x = v[k];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if ((threadIdx.x & 31) == 0 && x) atomicAdd(a.acc + k, x);
+  }
+}
+
+}  // namespace spa

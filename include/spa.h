@@ -1,0 +1,172 @@
+/*
+ * spa.h -- block-sparse long-context attention prefill on B200 (sm_100a).
+ *
+ * Two stages, both running entirely on the GPU:
+ *
+ *   sparse_prefill_plan   picks, for every 128-row query block, which keys
+ *                         outside the always-kept sink and local windows are
+ *                         attended to, and writes them as ascending index
+ *                         lists into a caller-owned workspace;
+ *   sparse_prefill_attn   runs causal softmax attention over exactly those
+ *                         keys (sink + selected + local) and writes O and,
+ *                         optionally, the row log-sum-exp.
+ *
+ * Selection modes
+ *   SPA_MODE_ANCHOR  AnchorAttention: Difference-Aware Sparse Attention with
+ *                    Stripe Granularity, Eq. (1)-(3): anchor x_a[i] = max score
+ *                    over the sink and local keys of row i; candidate key j of
+ *                    block b is kept iff mean_i(x_a[i]) - mean_i(q_i).k_j*scale
+ *                    <= theta (key-stripe granularity, block_k = 1).
+ *   SPA_MODE_SALE    SALE: Low-bit Estimation for Efficient Sparse Attention in
+ *                    Long-context LLM Prefilling, Sec. 3.2-3.4: S~ from 4-bit
+ *                    quantised Q and smoothed K; key block kb (block_k keys) is
+ *                    kept iff some row i and key j in kb have
+ *                    S~_ij >= ln(tau * el_i) + em_i, em/el being the max and the
+ *                    sum of exp(S~ - em) over the row's sink and local keys.
+ *   SPA_MODE_DENSE   no selection: every causal key (the "same kernel, dense"
+ *                    reference point for speedups).
+ *
+ * Geometry (all modes).  Query block b = rows [b*block_q, (b+1)*block_q) (the
+ * last one may be ragged).  Sink keys [0, sink).  Local window
+ * [ls_b, (b+1)*block_q), ls_b = max(0, (b+1)*block_q - local), causally cut
+ * per row.  Candidates C_b = [sink, ls_b).  Row i of block b attends to
+ * (sink u local u selected(b)) n {j <= i}.
+ *
+ * Tensors.  Q: bf16 [B, Hq, L, 128]; K, V: bf16 [B, Hkv, L, 128]; O: bf16
+ * [B, Hq, L, 128]; LSE: fp32 [B, Hq, L] (natural log).  Row-major, head_dim
+ * innermost, contiguous, device pointers, 16-byte aligned.  q head h reads kv
+ * head h / (Hq / Hkv) (grouped-query attention).
+ *
+ * Ownership.  The caller allocates and owns Q, K, V, O, LSE and the
+ * workspace; the library never allocates or frees device memory and keeps no
+ * state between calls.  Every call is asynchronous on the given stream except
+ * sparse_prefill_stats, which synchronises that stream.  A workspace written
+ * by sparse_prefill_plan stays valid for sparse_prefill_attn and
+ * sparse_prefill_stats until the next plan on the same workspace.  Two calls
+ * that share a workspace must not overlap on the GPU.
+ *
+ * Errors.  Argument, shape, alignment and workspace-size errors are returned
+ * synchronously, before anything is launched.  A failed launch returns
+ * SPA_ERR_CUDA.  Kernels never trap: a bounded wait that expires, or an index
+ * that fails a device-side check, sets a bit in the workspace error word and
+ * the kernel returns early; sparse_prefill_stats reports it (as
+ * SPA_ERR_TIMEOUT or SPA_ERR_INVALID) and the outputs of that call are
+ * undefined.
+ */
+#ifndef SPA_H_
+#define SPA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define SPA_API __attribute__((visibility("default")))
+#else
+#define SPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SPA_OK = 0,
+  SPA_ERR_INVALID = 1,      /* bad argument (null/misaligned pointer, bad size or value) */
+  SPA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head_dim != 128, causal == 0, step != 1, ...) */
+  SPA_ERR_WORKSPACE = 3,    /* workspace smaller than sparse_prefill_workspace_bytes() */
+  SPA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+  SPA_ERR_TIMEOUT = 5       /* a device-side bounded wait expired (reported by stats) */
+} spa_status;
+
+typedef enum {
+  SPA_MODE_ANCHOR = 0,
+  SPA_MODE_SALE = 1,
+  SPA_MODE_DENSE = 2
+} spa_mode;
+
+typedef struct {
+  int32_t batch;          /* B >= 0 (0 -> every call is a no-op) */
+  int32_t heads_q;        /* Hq >= 1 */
+  int32_t heads_kv;       /* Hkv >= 1, Hq % Hkv == 0 */
+  int32_t seq_len;        /* L >= 0; B*max(Hq,Hkv)*L < 2^31 */
+  int32_t head_dim;       /* must be 128 */
+  int32_t causal;         /* must be 1 */
+  int32_t block_q;        /* must be 128 */
+  int32_t block_k;        /* ANCHOR: 1 (key stripes); SALE: 16, 32, 64 or 128; DENSE: ignored */
+  int32_t sink;           /* >= 0; SALE: multiple of block_k */
+  int32_t local;          /* >= block_q, multiple of block_q */
+  int32_t step;           /* query blocks grouped per selection; must be 1 */
+  spa_mode mode;
+  float theta;            /* ANCHOR threshold, scaled-logit units; +inf keeps all; NaN invalid */
+  float tau;              /* SALE threshold on the relative score, 0 < tau <= 1 */
+  float softmax_scale;    /* > 0, or 0 for 1/sqrt(head_dim) */
+  uint32_t wait_limit_us; /* bound on every device-side wait; 0 -> 250,000 us */
+  uint32_t debug_flags;   /* 0 in normal use; SPA_DEBUG_* test hooks */
+} spa_params;
+
+/* Test hook: the attention kernel's MMA warp additionally waits on a barrier
+ * that nothing ever signals, so its bounded wait expires after wait_limit_us;
+ * the kernel then records SPA_ERR_TIMEOUT and returns without faulting. */
+#define SPA_DEBUG_STALL_ATTN 0x1u
+
+typedef struct {
+  uint32_t error_bits;       /* device error word: bit0 timeout, bit1 bad index */
+  uint32_t reserved;
+  int64_t query_blocks;      /* B * Hq * ceil(L / block_q) */
+  int64_t candidates;        /* sum over blocks of |C_b| (keys) */
+  int64_t kept_candidates;   /* sum over blocks of kept candidate keys */
+  int64_t kept_pairs;        /* sum over rows of |K_i|; kept FLOPs = 4 * head_dim * kept_pairs */
+  int64_t dense_pairs;       /* sum over rows of (i + 1): the causal dense count */
+} spa_stats;
+
+/* Bytes of device workspace sparse_prefill_plan/attn need for these params
+ * (closed form; 0 when the params are invalid).
+ *
+ * Workspace layout (byte offsets; A(x) rounds x up to a multiple of 256;
+ * NB = B * Hq * ceil(L / 128); blocks are ordered (b, h, qb)):
+ *   [0, 256)            header: uint32 error word at 0, 5 int64 counters at 8;
+ *   256                 counts: int32[NB], kept candidates of each block
+ *                       (keys in ANCHOR mode, key blocks in SALE mode);
+ *   A(256 + 4 * NB)     lists: int32, ascending.  The list of block (b, h, qb)
+ *                       starts at element (b * Hq + h) * P(nqb) + P(qb) with
+ *                       P(n) = sum_{q < n} max(0, (q + 1) * 128 - local - sink)
+ *                       in ANCHOR mode (key indices) and P(n) / block_k in
+ *                       SALE mode (key-block indices kb: keys [kb*block_k,
+ *                       (kb+1)*block_k)); capacity |C_b| keys per block;
+ *   after the lists     mode-specific scratch (opaque).
+ * DENSE mode uses only the header and the counts. */
+SPA_API size_t sparse_prefill_workspace_bytes(const spa_params* p);
+
+/* Selection.  Reads q, k; writes the index lists and counts into workspace.
+ * ANCHOR: anchor/pool kernel, pooled-score scan (tensor cores), compaction.
+ * SALE:   K mean, int4 quantisation of Q and K, sink-local statistics fused
+ *         with the int8 tensor-core block scan, compaction.
+ * DENSE:  only resets the workspace header. */
+SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const void* k,
+                               void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/* Attention over sink + selected + local keys (all causal keys in DENSE
+ * mode).  Reads q, k, v and the plan's lists; writes o and, when lse is not
+ * NULL, lse.  Records device-side errors in the workspace error word. */
+SPA_API spa_status sparse_prefill_attn(const spa_params* p, const void* q, const void* k,
+                               const void* v, void* workspace, size_t workspace_bytes,
+                               void* o, float* lse, cudaStream_t stream);
+
+/* Reduces the plan's counts into *out (host pointer) and synchronises the
+ * stream.  Returns SPA_ERR_TIMEOUT / SPA_ERR_INVALID when the error word is
+ * set, after filling *out. */
+SPA_API spa_status sparse_prefill_stats(const spa_params* p, const void* workspace,
+                                size_t workspace_bytes, spa_stats* out,
+                                cudaStream_t stream);
+
+/* Static string for a status code. */
+SPA_API const char* sparse_prefill_status_string(spa_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPA_H_ */

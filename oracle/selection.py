@@ -119,6 +119,43 @@ def anchor_block(qh: np.ndarray, kh: np.ndarray, qb: int, *, bq: int, sink: int,
                        xbar_a=xbar_a, qbar=qbar, sbar=sbar)
 
 
+def anchor_head(qh: np.ndarray, kh: np.ndarray, blocks, *, bq: int, sink: int, local: int,
+                theta: float, scale: float = 0.0):
+    """``anchor_block`` for several blocks of one head, the pooled scores of all
+    of them taken with a single matrix product avgpool(Q)_blocks K^T.
+
+    Returns {qb: AnchorBlock}; equal to calling ``anchor_block`` per block.
+    """
+    L, d = qh.shape
+    sc = default_scale(d, scale)
+    blocks = list(blocks)
+    out = {}
+    qbars = []
+    for qb in blocks:
+        geo = block_geometry(qb, L, bq, sink, local)
+        qbars.append(qh[geo.row_lo:geo.row_hi].mean(axis=0))
+    cand_hi_max = max((block_geometry(qb, L, bq, sink, local).cand_hi for qb in blocks), default=sink)
+    cand_all = np.arange(sink, max(sink, cand_hi_max))
+    sbar_all = (np.stack(qbars) @ kh[cand_all].T) * sc if blocks else None
+    for n, qb in enumerate(blocks):
+        geo = block_geometry(qb, L, bq, sink, local)
+        rows = np.arange(geo.row_lo, geo.row_hi)
+        slk = sink_local_keys(geo, sink)
+        s = (qh[rows] @ kh[slk].T) * sc
+        causal = slk[None, :] <= rows[:, None]
+        x_a = np.where(causal, s, -np.inf).max(axis=1)
+        xbar_a = float(x_a.mean())
+        cand = np.arange(geo.cand_lo, geo.cand_hi)
+        sbar = sbar_all[n, : cand.size]
+        diff = xbar_a - sbar
+        with np.errstate(invalid="ignore"):
+            margin = theta - diff
+        keep = diff <= theta
+        out[qb] = AnchorBlock(kept=cand[keep], cand=cand, margin=margin, x_a=x_a,
+                              xbar_a=xbar_a, qbar=qbars[n], sbar=sbar)
+    return out
+
+
 # ---------------------------------------------------------------------------
 # SALE: 4-bit estimate + Relative Attention Score block selection
 # ---------------------------------------------------------------------------

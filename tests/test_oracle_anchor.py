@@ -162,3 +162,14 @@ def test_handmade_exact_ties_keep():
                                 local=g["local"], theta=case["theta"], scale=tc["scale"])
         assert blk.xbar_a == case["xbar"]
         np.testing.assert_array_equal(blk.kept, _ranges_to_keys(case["kept_ranges"]), err_msg=str(case))
+
+
+def test_anchor_head_equals_per_block():
+    w, qh, kh, _ = _small_case(L=1100)
+    blocks = [0, 1, 2, 5, 8]
+    many = osel.anchor_head(qh, kh, blocks, bq=w.block_q, sink=w.sink, local=w.local, theta=2.7)
+    for qb in blocks:
+        one = osel.anchor_block(qh, kh, qb, bq=w.block_q, sink=w.sink, local=w.local, theta=2.7)
+        np.testing.assert_array_equal(many[qb].kept, one.kept)
+        np.testing.assert_allclose(many[qb].margin, one.margin, atol=1e-12, rtol=0)
+        assert many[qb].xbar_a == one.xbar_a
