@@ -72,6 +72,8 @@ def _load():
     lib.sparse_prefill_attn.restype = ctypes.c_int
     lib.sparse_prefill_stats.argtypes = [P, vp, sz, ctypes.POINTER(SpaStats), vp]
     lib.sparse_prefill_stats.restype = ctypes.c_int
+    lib.sparse_prefill_plan_static.argtypes = [P, vp, vp, vp, vp, sz, vp, vp]
+    lib.sparse_prefill_plan_static.restype = ctypes.c_int
     lib.sparse_prefill_status_string.argtypes = [ctypes.c_int]
     lib.sparse_prefill_status_string.restype = ctypes.c_char_p
     return lib
@@ -144,6 +146,15 @@ def sparse_prefill_stats(params: SpaParams, workspace, workspace_bytes=None, str
     st = int(_lib.sparse_prefill_stats(ctypes.byref(params), _ptr(workspace), wb,
                                        ctypes.byref(out), _stream(stream)))
     return st, out
+
+
+def sparse_prefill_plan_static(params: SpaParams, q, k, counts, lists, lists_elems=None,
+                               error_word=None, stream=None) -> int:
+    """Allocation-free ANCHOR plan: scratch in the library's fixed device array."""
+    n = lists.numel() if lists_elems is None else int(lists_elems)
+    return int(_lib.sparse_prefill_plan_static(ctypes.byref(params), _ptr(q), _ptr(k),
+                                               _ptr(counts), _ptr(lists), n, _ptr(error_word),
+                                               _stream(stream)))
 
 
 def sparse_prefill_status_string(status: int) -> str:

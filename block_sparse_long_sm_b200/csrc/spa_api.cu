@@ -4,6 +4,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -372,6 +373,136 @@ SPA_API spa_status sparse_prefill_stats(const spa_params* p, const void* workspa
   out->dense_pairs = (int64_t)v[4];
   if (errw & kErrTimeout) return SPA_ERR_TIMEOUT;
   if (errw & kErrBadIndex) return SPA_ERR_INVALID;
+  return SPA_OK;
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the ANCHOR-mode plan.
+//
+// Some callers cannot hand this library a workspace: plugin hosts whose
+// enqueue step may not allocate device memory, serving stacks that reserve
+// their whole memory budget at start-up and own every byte afterwards, and
+// hot paths that must not call cudaMalloc because it can synchronise the
+// device.  For them the selection's scratch (workspace header, anchor means,
+// pooled queries, key bitmask) lives in the fixed array below; the caller
+// still provides the inputs (Q, K) and the outputs (counts, lists).
+//
+// The array is kStaticScratchBytes per GPU, held by every GPU that loads the
+// library until the process exits.  All calls share it and it keeps the last
+// call's contents, so two calls that overlap on the GPU (different streams,
+// different threads) race; callers must serialise them.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = SPA_STATIC_SCRATCH_BYTES;
+__device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mutex;
+void* g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_static_scratch on the current device, looked up once
+// per device (the host-side name is only a stand-in, not a device address).
+void* static_scratch_ptr() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(g_static_mutex);
+  if (!g_static_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
+    g_static_ptr[dev] = ptr;
+  }
+  return g_static_ptr[dev];
+}
+
+struct StaticLayout {
+  size_t xbar, qbar, mask, total;
+};
+
+StaticLayout static_layout(const spa_params* p, const Layout& lo) {
+  StaticLayout s;
+  size_t off = kHeaderBytes;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align_up(off + bytes);
+    return at;
+  };
+  s.xbar = take(lo.nb * 4);
+  s.qbar = take((size_t)2 * lo.nb * 128 * 2);
+  s.mask = take((size_t)lo.nb * lo.nwords * 4);
+  s.total = off;
+  (void)p;
+  return s;
+}
+
+}  // namespace
+
+extern "C" {
+
+SPA_API spa_status sparse_prefill_plan_static(const spa_params* p, const void* q, const void* k,
+                                              int32_t* counts, int32_t* lists,
+                                              size_t lists_elems, uint32_t* error_word,
+                                              cudaStream_t stream) {
+  spa_status st = validate(p);
+  if (st != SPA_OK) return st;
+  if (p->mode != SPA_MODE_ANCHOR) return SPA_ERR_UNSUPPORTED;
+  const Layout lo = layout_of(p);
+  const StaticLayout sl = static_layout(p, lo);
+  if (sl.total > kStaticScratchBytes) return SPA_ERR_UNSUPPORTED;
+  const int B = p->batch, Hq = p->heads_q, Hkv = p->heads_kv, L = p->seq_len;
+  if (B == 0 || L == 0) return SPA_OK;
+  if (!q || !k || !counts || !aligned16(q) || !aligned16(k) ||
+      (reinterpret_cast<uintptr_t>(counts) & 3u))
+    return SPA_ERR_INVALID;
+  const long long list_elems = (long long)B * Hq * lo.list_per_head;
+  if ((size_t)list_elems > lists_elems) return SPA_ERR_WORKSPACE;
+  if (list_elems > 0 && (!lists || (reinterpret_cast<uintptr_t>(lists) & 3u)))
+    return SPA_ERR_INVALID;
+  uint8_t* ws = static_cast<uint8_t*>(static_scratch_ptr());
+  if (!ws) return SPA_ERR_CUDA;
+  // the header (error word) must start at zero; the rest is fully rewritten
+  if (cudaMemsetAsync(ws, 0, kHeaderBytes, stream) != cudaSuccess) return SPA_ERR_CUDA;
+  uint32_t* err = reinterpret_cast<uint32_t*>(ws);
+  const float scale = eff_scale(p);
+  const long long BH = (long long)B * Hq, BKV = (long long)B * Hkv;
+  CUtensorMap tq, tk, tqbar;
+  if (!map_2d(&tq, kBF16, 2, q, 128, BH * L, 64, 128, kSW128) ||
+      !map_2d(&tk, kBF16, 2, k, 128, BKV * L, 64, 128, kSW128) ||
+      !map_3d(&tqbar, kBF16, 2, ws + sl.qbar, 128, lo.nqb, 2 * BH, 64, 128, kSW128))
+    return SPA_ERR_CUDA;
+  PoolArgs pa{B, Hq, Hkv, L, lo.nqb, lo.group, p->sink, p->local, scale,
+              reinterpret_cast<float*>(ws + sl.xbar),
+              reinterpret_cast<__nv_bfloat16*>(ws + sl.qbar), err, wait_ns(p)};
+  if (set_smem(anchor_pool_kernel, kPoolSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
+  anchor_pool_kernel<<<(unsigned)lo.nb, kPoolThreads, kPoolSmemBytes, stream>>>(tq, tk, pa);
+  if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
+  const int nmt = (lo.nqb + 127) / 128;
+  const int key_end = std::max(0, lo.nqb * 128 - p->local);
+  const int kt0 = p->sink / 128;
+  const int kt_end = (key_end + 127) / 128;
+  const int nchunk = key_end > p->sink
+                         ? (kt_end - kt0 + kScanTilesPerChunk - 1) / kScanTilesPerChunk
+                         : 0;
+  if (nchunk > 0) {
+    ScanArgs sa{B, Hq, Hkv, L, lo.nqb, lo.group, p->sink, p->local, p->theta,
+                reinterpret_cast<const float*>(ws + sl.xbar),
+                reinterpret_cast<uint32_t*>(ws + sl.mask), lo.nwords, err, wait_ns(p)};
+    if (set_smem(stripe_scan_kernel, kScanSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
+    stripe_scan_kernel<<<dim3(nchunk, nmt, (unsigned)BH), kScanThreads, kScanSmemBytes,
+                         stream>>>(tqbar, tk, sa);
+    if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
+  }
+  CompactArgs ca{(int)lo.nb, lo.nqb, L, p->sink, p->local, 1,
+                 reinterpret_cast<const uint32_t*>(ws + sl.mask), lo.nwords, lists,
+                 lo.list_per_head, lo.cap_a, counts};
+  compact_kernel<<<(unsigned)lo.nb, kCompactThreads, 0, stream>>>(ca);
+  if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
+  if (error_word &&
+      cudaMemcpyAsync(error_word, err, sizeof(uint32_t), cudaMemcpyDeviceToDevice, stream) !=
+          cudaSuccess)
+    return SPA_ERR_CUDA;
   return SPA_OK;
 }
 

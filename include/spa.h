@@ -162,6 +162,43 @@ SPA_API spa_status sparse_prefill_stats(const spa_params* p, const void* workspa
                                 size_t workspace_bytes, spa_stats* out,
                                 cudaStream_t stream);
 
+/* Allocation-free selection (ANCHOR mode only).  The paper has no
+ * counterpart: this entry point exists for callers that cannot give the
+ * library a workspace -- plugin hosts whose enqueue step may not allocate
+ * device memory, serving stacks that reserve their whole memory budget at
+ * start-up, and hot paths that must not call cudaMalloc because it can
+ * synchronise the device.  It computes exactly what sparse_prefill_plan
+ * computes, but the scratch (header, anchor means, pooled queries, key
+ * bitmask) lives in a fixed device array of SPA_STATIC_SCRATCH_BYTES inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits.  Nothing is allocated or freed.
+ *
+ *   q, k        inputs as for sparse_prefill_plan (device, 16-byte aligned);
+ *   counts      output, device int32[B*Hq*ceil(L/128)], blocks in (b, h, qb) order;
+ *   lists       output, device int32[lists_elems]: the block lists at the
+ *               offsets documented for the workspace's list region, relative
+ *               to `lists` (B*Hq*P(nqb) elements are needed);
+ *   error_word  optional device uint32 that receives the device error word
+ *               (bit0 timeout, bit1 bad index) after the call; may be NULL.
+ *
+ * Returns SPA_ERR_UNSUPPORTED when the mode is not ANCHOR or when the scratch
+ * these params need exceeds SPA_STATIC_SCRATCH_BYTES (about B*Hq*L*L/1024
+ * bytes of bitmask plus 516 bytes per query block; 32 q heads fit up to
+ * L = 32768), SPA_ERR_WORKSPACE when lists_elems is too small, and the same
+ * argument errors as sparse_prefill_plan, all before any launch.
+ *
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture.  All calls share the array and it keeps the last
+ * call's contents (the header is cleared on every call); calls that overlap
+ * on the GPU -- on different streams or from different threads -- race and
+ * must be serialised by the caller. */
+#define SPA_STATIC_SCRATCH_BYTES ((size_t)48 << 20)
+SPA_API spa_status sparse_prefill_plan_static(const spa_params* p, const void* q, const void* k,
+                                              int32_t* counts, int32_t* lists,
+                                              size_t lists_elems, uint32_t* error_word,
+                                              cudaStream_t stream);
+
 /* Static string for a status code. */
 SPA_API const char* sparse_prefill_status_string(spa_status s);
 
