@@ -224,7 +224,25 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_load_2d(s_q, &tm_q, bar_q, 0, qrow);
       tma_load_2d(s_q + kHalfBytes, &tm_q, bar_q, 64, qrow);
     }
+    // Indices of a gathered tile: this lane's four rows (padding rows repeat
+    // the tile's first key).  They are fetched one tile ahead so that the
+    // global-load latency overlaps the wait for a free stage.
+    auto fetch = [&](int t, int (&j)[4], int& first) {
+      const TileDesc td = tile_desc(it, t);
+      if (!td.gather) return;
+      first = sel_key(a, it, td.key0);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int row = lane * 4 + r;
+        j[r] = row < td.valid ? sel_key(a, it, td.key0 + row) : first;
+      }
+    };
+    int nj[4] = {0, 0, 0, 0}, nfirst = 0;
+    if (T > 0) fetch(0, nj, nfirst);
     for (int t = 0; t < T; ++t) {
+      int j[4] = {nj[0], nj[1], nj[2], nj[3]};
+      const int first = nfirst;
+      if (t + 1 < T) fetch(t + 1, nj, nfirst);
       const int st = t % kAttnStages;
       if (t >= kAttnStages) {
         if (!warp_wait(bar_empty(st), ((t / kAttnStages) - 1) & 1, wc)) break;
@@ -241,20 +259,18 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
           tma_load_2d(s_v(st) + kHalfBytes, &tm_v, vf, 64, kv_row0 + td.key0);
         }
       } else {
-        // indices of this lane's four rows (padding rows repeat the first key)
-        int j[4];
-        const int first = sel_key(a, it, td.key0);
+        bool bad = false;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          const int row = lane * 4 + r;
-          j[r] = row < td.valid ? sel_key(a, it, td.key0 + row) : first;
           if (j[r] < 0 || j[r] >= a.L) {
-            atomicOr(a.err, kErrBadIndex);
+            bad = true;
             j[r] = 0;
           }
         }
+        if (bad) atomicOr(a.err, kErrBadIndex);
         const int last = __shfl_sync(0xffffffffu, j[3], 31);
-        const bool contiguous = (td.valid == 128) && (last - first == 127);
+        const bool contiguous = (td.valid == 128) && (last - first == 127) && first >= 0 &&
+                                first < a.L && last < a.L;
         if (lane == 0) {
           mbar_arrive_expect_tx(kf, kTileBytes);
           mbar_arrive_expect_tx(vf, kTileBytes);
@@ -353,17 +369,26 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
 
       const TileDesc td = tile_desc(it, t);
       const int limit = td.causal ? min(td.valid, r + 1) : td.valid;
-      float mx = -INFINITY;
+      // row max with eight independent accumulators (no serial chain)
+      float mxv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mxv[u] = -INFINITY;
+      if (limit < 128) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            if (c * 32 + e >= limit) sr[c][e] = __float_as_uint(-INFINITY);
+          }
+        }
+      }
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          float v = __uint_as_float(sr[c][e]);
-          if (c * 32 + e >= limit) v = -INFINITY;
-          sr[c][e] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
-        }
+        for (int e = 0; e < 32; ++e) mxv[e & 7] = fmaxf(mxv[e & 7], __uint_as_float(sr[c][e]));
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
+                             fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
       const float mx2 = mx * sl2;
       const bool grow = mx2 > m_used + 8.0f;
       if (t == 0) {
@@ -392,18 +417,20 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tm_q,
       // p = 2^(s * scale * log2 e - m); masked entries give 0
       const float neg_m = -m_used;
       uint32_t pk[2][32];
-      float psum = 0.f;
+      float ps[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ps[u] = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][e]), sl2, neg_m));
           const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m));
-          psum += p0 + p1;
+          ps[(e >> 1) & 7] += p0 + p1;
           pk[c >> 1][(c & 1) * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
         }
       }
-      lsum += psum;
+      lsum += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       // P_b is free once the PV of tile t-2 has completed
       if (t >= 2 && !(ok = warp_wait(bar_pvdone0 + 8u * b, ((t - 2) >> 1) & 1, wc))) break;
       tc_fence_after();
