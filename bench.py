@@ -110,6 +110,28 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def _kernel_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for name in ("attn.cuh", "ptx.cuh"):
+        with open(os.path.join(ROOT, "block_sparse_long_sm_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def _recorded_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    record, only if the kernel source is the one the counters were taken on."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)["sparse_attn_kernel"]
+    except Exception:
+        return None
+    if rec.get("source_sha256") != _kernel_source_hash() or rec.get("workload") != workload:
+        return None
+    return rec.get("bytes_per_launch")
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -117,9 +139,10 @@ def _dist():
     return world, rank, local
 
 
-def oracle_sample(w: Workload, inp, theta: float, n_blocks: int = 3):
-    """CPU oracle on a bounded sample: anchor selection + sparse attention for the
-    last ``n_blocks`` query blocks of q head 0 (every row of those blocks)."""
+def oracle_sample(w: Workload, inp, theta: float, n_rows: int = 256):
+    """CPU oracle on a bounded sample: anchor selection for the query blocks that
+    hold the last ``n_rows`` rows of q head 0, then fp64 sparse attention for
+    those rows (the longest rows of the layer)."""
     from oracle import attention as oatt
     from oracle import selection as osel
     from workloads import bf16_bits_to_f32
@@ -127,17 +150,19 @@ def oracle_sample(w: Workload, inp, theta: float, n_blocks: int = 3):
     kh = bf16_bits_to_f32(inp.k[0, 0]).astype(np.float64)
     vh = bf16_bits_to_f32(inp.v[0, 0]).astype(np.float64)
     L = w.seq_len
-    nqb = (L + 127) // 128
-    blocks = list(range(nqb - n_blocks, nqb))
+    rows = list(range(max(0, L - n_rows), L))
+    blocks = sorted({i // 128 for i in rows})
     t0 = time.perf_counter()
     sel = {qb: osel.anchor_block(qh, kh, qb, bq=128, sink=w.sink, local=w.local,
                                  theta=theta).kept for qb in blocks}
-    rows = range(blocks[0] * 128, L)
     oatt.attend_rows(qh, kh, vh, rows, lambda i: i // 128, lambda b: sel[b], bq=128,
                      sink=w.sink, local=w.local)
     dt = time.perf_counter() - t0
-    pairs = sum(oatt.kept_pairs_block(qb, L, bq=128, sink=w.sink, local=w.local,
-                                      n_selected=len(sel[qb])) for qb in blocks)
+    pairs = 0
+    for i in rows:
+        qb = i // 128
+        ls = max(0, (qb + 1) * 128 - w.local)
+        pairs += min(w.sink, ls) + (i + 1 - ls) + len(sel[qb])
     flops = 4 * 128 * pairs
     cores = len(os.sched_getaffinity(0))
     try:
@@ -147,8 +172,8 @@ def oracle_sample(w: Workload, inp, theta: float, n_blocks: int = 3):
     except Exception:
         pass
     return dict(value=flops / dt / 1e12, unit=UNIT, cores=cores, kind="oracle",
-                sample=f"q head 0, last {n_blocks} query blocks ({len(rows)} rows) of "
-                       f"{w.name}: anchor selection + fp64 sparse attention; {dt:.1f} s",
+                sample=f"q head 0, last {len(rows)} rows of {w.name} (their query blocks' "
+                       f"anchor selection + fp64 sparse attention); {dt:.1f} s",
                 seconds=dt, flops=flops)
 
 
@@ -158,17 +183,18 @@ def run_reference(args, w: Workload):
         return
     inp = generate(w, kv_groups=[0])
     vals = []
-    for _ in range(args.warmup_ref):
-        oracle_sample(w, inp, args.theta, n_blocks=1)
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, args.theta, n_rows=16)
     for _ in range(args.steps):
-        vals.append(oracle_sample(w, inp, args.theta, n_blocks=1))
+        vals.append(oracle_sample(w, inp, args.theta, n_rows=16))
     v = statistics.median(x["value"] for x in vals)
     cb = dict(vals[-1])
     cb["value"] = v
     for key in ("seconds", "flops"):
         cb.pop(key, None)
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": None,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": statistics.median(x["seconds"] for x in vals) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": _config(w, args),
             "cpu_baseline": cb, "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -180,7 +206,9 @@ def _config(w: Workload, args):
     return {"workload": w.name, "batch": w.batch, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
             "seq_len": w.seq_len, "head_dim": 128, "causal": True, "mode": args.mode,
             "theta": args.theta, "sink": w.sink, "local": w.local, "block_q": 128,
-            "l2": "inputs (1.5 GB) larger than L2; no flush",
+            "l2": f"inputs ({2 * 128 * w.seq_len * w.batch * (w.heads_q + 2 * w.heads_kv) / 1e9:.2f} GB) "
+                  + ("larger than L2 (126 MB); no flush" if w.seq_len * w.batch * (w.heads_q + 2 * w.heads_kv) * 256 > 126e6
+                     else "smaller than L2"),
             "parallelism": "independent layer per GPU"}
 
 
@@ -194,7 +222,6 @@ def main():
     ap.add_argument("--theta", type=float, default=5.0)
     ap.add_argument("--config", default=C2_LLAMA_128K.name, choices=sorted(CONFIGS))
     ap.add_argument("--no-extras", action="store_true", help="skip SALE/dense/e2e/cpu legs")
-    ap.add_argument("--warmup-ref", type=int, default=0)
     args = ap.parse_args()
     w = CONFIGS[args.config]
     if args.impl == "reference":
@@ -286,7 +313,8 @@ def main():
             "kept_flops_per_layer": flops_step,
             "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel",
                          "achieved": achieved, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
-                         "frac": achieved / peaks["bf16_sus"], "traffic": None,
+                         "frac": achieved / peaks["bf16_sus"],
+                         "traffic": _recorded_traffic(w.name),
                          "peak_source": f"{peaks['src']} bf16 dense, sustained (kernel timed inside a long loop)"},
             "clocks": clk.summary(),
             "gpu_launches": launches,
@@ -350,7 +378,6 @@ def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, st
     sale_attn = timed(lambda: spa.check(spa.sparse_prefill_attn(ps, q, k, v, wss, o, None, stream=stream)))
     st, ss = spa.sparse_prefill_stats(ps, wss, stream=stream)
     sflops = spa.kept_flops(ss)
-    int_ops = 2 * 128 * (ss.candidates * 128)    # scan: every candidate (row, key) pair, per block row
     out["sale"] = {"tau": w.tau, "block_k": w.block_k, "plan_ms": sale_plan, "attn_ms": sale_attn,
                    "kept_fraction": ss.kept_pairs / ss.dense_pairs,
                    "kept_tflops": sflops / ((sale_plan + sale_attn) / 1e3) / 1e12}
@@ -382,7 +409,7 @@ def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, st
     # CPU oracle on a bounded sample (same metric and unit)
     if int(os.environ.get("WORLD_SIZE", "1")) == 1:
         inp = generate(w, kv_groups=[0])
-        cb = oracle_sample(w, inp, args.theta, n_blocks=2)
+        cb = oracle_sample(w, inp, args.theta, n_rows=256)
         cb.pop("seconds", None)
         cb.pop("flops", None)
         out["cpu_baseline"] = cb

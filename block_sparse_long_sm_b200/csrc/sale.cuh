@@ -89,13 +89,22 @@ __global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
 // ---------------------------------------------------------------------------
 // fused sink-local statistics + block scan
 // ---------------------------------------------------------------------------
+// Tiles are 128 keys (M = 128 rows, N = 128, K = 128 int8 in four MMAs) so
+// that four TMEM accumulators (128 columns each) let the tensor core run up
+// to three tiles ahead of the epilogue.  Warps 2-9 form the epilogue: warp w
+// reads TMEM lanes 32*(w%4).. and columns [64*h, 64*h+64) of each tile,
+// h = (w-2)/4.  The per-key-block scales of the kv head are staged in shared
+// memory once per CTA.
 constexpr int kSaleThreads = 320;            // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
-constexpr int kSaleStages = 3;
+constexpr int kSaleStages = 4;
+constexpr int kSaleBufs = 4;                 // TMEM accumulators of 128 columns
 constexpr uint32_t kQ8Bytes = 128u * 128u;   // 128 rows x 128 int8
-constexpr uint32_t kK8Bytes = 256u * 128u;   // 256 rows x 128 int8
+constexpr uint32_t kK8Bytes = 128u * 128u;   // 128 keys x 128 int8
 constexpr int kMaxGroupWords = 512;          // candidate 16-key groups / 32 (L <= 262144)
-constexpr uint32_t kSaleSmemBytes =
-    1024u + kQ8Bytes + kSaleStages * kK8Bytes + 512u + kMaxGroupWords * 4u + 128u * 16u;
+constexpr int kMaxScales = 16384;            // key blocks per head (L / bk <= 16384)
+constexpr uint32_t kSaleSmemBytes = 1024u + kQ8Bytes + kSaleStages * kK8Bytes + 1024u +
+                                    kMaxGroupWords * 4u + 128u * 16u + kMaxScales * 4u;
+constexpr uint32_t kIdescI8N128 = make_idesc(2, 1, 128, 128, 0, 0);
 
 struct SaleArgs {
   int B, Hq, Hkv, L, nqb, group;
@@ -121,16 +130,17 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
   uint8_t* bar_area = smem + kQ8Bytes + kSaleStages * kK8Bytes;
   const uint32_t b0 = smem_u32(bar_area);
   const uint32_t bar_q = b0;
-  auto bar_full = [&](int s) { return b0 + 8u * (1 + s); };
-  auto bar_empty = [&](int s) { return b0 + 8u * (1 + kSaleStages + s); };
-  const uint32_t bar_sfull0 = b0 + 8u * (1 + 2 * kSaleStages);
-  const uint32_t bar_sfree0 = bar_sfull0 + 16u;
-  const uint32_t bar_drain = bar_sfull0 + 32u;
-  const uint32_t bar_stat = bar_sfull0 + 40u;     // both column halves of every row posted
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 8 * (1 + 2 * kSaleStages) + 48);
+  auto bar_full = [&](int st) { return b0 + 8u * (1 + st); };
+  auto bar_empty = [&](int st) { return b0 + 8u * (1 + kSaleStages + st); };
+  auto bar_sfull = [&](int bb) { return b0 + 8u * (1 + 2 * kSaleStages + bb); };
+  auto bar_sfree = [&](int bb) { return b0 + 8u * (1 + 2 * kSaleStages + kSaleBufs + bb); };
+  const uint32_t bar_drain = b0 + 8u * (1 + 2 * kSaleStages + 2 * kSaleBufs);
+  const uint32_t bar_stat = bar_drain + 8u;       // both column halves of every row posted
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 512);
   volatile uint32_t* abort_flag = tmem_holder + 1;
-  uint32_t* gflags = reinterpret_cast<uint32_t*>(bar_area + 512);       // candidate group flags
-  float* part = reinterpret_cast<float*>(gflags + kMaxGroupWords);      // [128][4]: m,l of 2 halves
+  uint32_t* gflags = reinterpret_cast<uint32_t*>(bar_area + 1024);    // candidate group flags
+  float* part = reinterpret_cast<float*>(gflags + kMaxGroupWords);    // [128][4]: m,l of 2 halves
+  float* cscale = part + 128 * 4;                                     // sq*sk*scale per key block
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int x = blockIdx.x;
@@ -141,29 +151,27 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
   const int le = min(row0 + 128, a.L);
   const int ls = max(0, row0 + 128 - a.local);
   const int sink_end = min(a.sink, ls);
-  // tiles of 256 keys: sink, local (statistics), then candidates (scan)
-  const int n_sink_t = (sink_end + 255) / 256;
-  const int n_loc_t = (le - ls + 255) / 256;
+  const int n_sink_t = (sink_end + 127) / 128;
+  const int n_loc_t = (le - ls + 127) / 128;
   const int cand_lo = a.sink, cand_hi = max(a.sink, ls);
-  const int n_cand_t = (cand_hi - cand_lo + 255) / 256;
+  const int n_cand_t = (cand_hi - cand_lo + 127) / 128;
   const int n_stat_t = n_sink_t + n_loc_t;
   const int T = n_stat_t + n_cand_t;
-  const int n_groups = (cand_hi - cand_lo) / 16;
   auto tile_key0 = [&](int t) {
-    if (t < n_sink_t) return t * 256;
-    if (t < n_stat_t) return ls + (t - n_sink_t) * 256;
-    return cand_lo + (t - n_stat_t) * 256;
+    if (t < n_sink_t) return t * 128;
+    if (t < n_stat_t) return ls + (t - n_sink_t) * 128;
+    return cand_lo + (t - n_stat_t) * 128;
   };
 
   if (threadIdx.x == 0) {
     mbar_init(bar_q, 1);
-    for (int s = 0; s < kSaleStages; ++s) {
-      mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
+    for (int st = 0; st < kSaleStages; ++st) {
+      mbar_init(bar_full(st), 1);
+      mbar_init(bar_empty(st), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_sfull0 + 8u * i, 1);
-      mbar_init(bar_sfree0 + 8u * i, 256);
+    for (int i = 0; i < kSaleBufs; ++i) {
+      mbar_init(bar_sfull(i), 1);
+      mbar_init(bar_sfree(i), 256);
     }
     mbar_init(bar_drain, 1);
     mbar_init(bar_stat, 256);
@@ -171,6 +179,12 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
     fence_barrier_init();
   }
   for (int i = threadIdx.x; i < kMaxGroupWords; i += blockDim.x) gflags[i] = 0u;
+  {
+    const float cq = a.sq[(long long)bh * a.nqb + qb] * a.scale;
+    const int nkb_used = min(a.nkb, (le + a.bk - 1) / a.bk);
+    const float* skp = a.sk + (long long)bkv * a.nkb;
+    for (int i = threadIdx.x; i < nkb_used; i += blockDim.x) cscale[i] = cq * skp[i];
+  }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
@@ -204,16 +218,18 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
     if (lane == 0) {
       bool ok = mbar_wait(bar_q, 0, wc);
       for (int t = 0; ok && t < T; ++t) {
-        const int st = t % kSaleStages, bb = t & 1;
+        const int st = t % kSaleStages, bb = t % kSaleBufs;
         if (!(ok = mbar_wait(bar_full(st), (t / kSaleStages) & 1, wc))) break;
-        if (t >= 2 && !(ok = mbar_wait(bar_sfree0 + 8u * bb, ((t - 2) >> 1) & 1, wc))) break;
+        if (t >= kSaleBufs &&
+            !(ok = mbar_wait(bar_sfree(bb), ((t / kSaleBufs) - 1) & 1, wc)))
+          break;
         tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-          mma_i8_ss(tmem + 256u * bb, smem_desc_sw128(s_q + ks * 32u, 16),
-                    smem_desc_sw128(s_k(st) + ks * 32u, 16), kIdescI8, ks > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_i8_ss(tmem + 128u * bb, smem_desc_sw128(s_q + kk * 32u, 16),
+                    smem_desc_sw128(s_k(st) + kk * 32u, 16), kIdescI8N128, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar_sfull0 + 8u * bb);
+        mma_commit(bar_sfull(bb));
         mma_commit(bar_empty(st));
       }
       mma_commit(bar_drain);
@@ -221,48 +237,39 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
     }
     __syncwarp();
   } else {
-    const int ew = warp - 2;                 // 0..7
     const int quad = warp & 3;               // TMEM lane quadrant
-    const int half = ew >> 2;                // columns [128*half, 128*half + 128)
+    const int half = (warp - 2) >> 2;        // columns [64*half, 64*half + 64)
     const int r = quad * 32 + lane;
     const int row = row0 + r;
     const bool row_valid = row < a.L;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const float cq = a.sq[(long long)bh * a.nqb + qb] * a.scale;
-    const float* skp = a.sk + (long long)bkv * a.nkb;
     float m = -INFINITY, l = 0.f, thr = INFINITY;
-    bool ok = true;
     for (int t = 0; t < T; ++t) {
-      const int bb = t & 1;
-      if (!(ok = warp_wait(bar_sfull0 + 8u * bb, (t >> 1) & 1, wc))) break;
+      const int bb = t % kSaleBufs;
+      if (!warp_wait(bar_sfull(bb), (t / kSaleBufs) & 1, wc)) break;
       tc_fence_after();
-      uint32_t sr[4][32];
+      uint32_t sr[2][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
-        tmem_ld32(tmem + lane_off + 256u * bb + 128u * half + 32u * c, sr[c]);
+      for (int c = 0; c < 2; ++c) tmem_ld32(tmem + lane_off + 128u * bb + 64u * half + 32u * c, sr[c]);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar_sfree0 + 8u * bb);
-      const int key0 = tile_key0(t) + 128 * half;
+      mbar_arrive(bar_sfree(bb));
+      const int key0 = tile_key0(t) + 64 * half;
       if (t < n_stat_t) {
         // S~ over the causal sink-local keys of this row
-        int limit;
-        if (t < n_sink_t) limit = sink_end - key0;
-        else limit = min(le - key0, row - key0 + 1);
-        limit = max(0, min(limit, 128));
+        int limit = (t < n_sink_t) ? sink_end - key0 : min(le - key0, row - key0 + 1);
+        limit = max(0, min(limit, 64));
         float tm = -INFINITY;
-        float sv[4][32];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int col = c * 32 + e;
-            const int key = key0 + col;
-            const float sk = skp[min(key, a.L - 1) / a.bk];
             const float v = col < limit
-                                ? static_cast<float>(static_cast<int>(sr[c][e])) * (cq * sk)
+                                ? static_cast<float>(static_cast<int>(sr[c][e])) *
+                                      cscale[min(key0 + col, a.L - 1) / a.bk]
                                 : -INFINITY;
-            sv[c][e] = v;
+            sr[c][e] = __float_as_uint(v);
             tm = fmaxf(tm, v);
           }
         }
@@ -270,10 +277,10 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
           const float mn = fmaxf(m, tm);
           float acc = 0.f;
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc += expf(sv[c][e] - mn);
-          l = l * expf(m - mn) + acc;
+            for (int e = 0; e < 32; ++e) acc += __expf(__uint_as_float(sr[c][e]) - mn);
+          l = l * __expf(m - mn) + acc;
           m = mn;
         }
         if (t == n_stat_t - 1) {
@@ -281,7 +288,7 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
           part[r * 4 + half * 2 + 0] = m;
           part[r * 4 + half * 2 + 1] = l;
           mbar_arrive(bar_stat);
-          if (!(ok = warp_wait(bar_stat, 0, wc))) break;
+          if (!warp_wait(bar_stat, 0, wc)) break;
           const float m0 = part[r * 4 + 0], l0 = part[r * 4 + 1];
           const float m1 = part[r * 4 + 2], l1 = part[r * 4 + 3];
           const float em = fmaxf(m0, m1);
@@ -293,29 +300,26 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
         // candidate tile: one flag per 16-key group (groups never straddle ls)
         uint32_t gbits = 0;
 #pragma unroll
-        for (int g = 0; g < 8; ++g) {
-          const int key = key0 + 16 * g;
-          int mx = INT_MIN;
+        for (int g = 0; g < 4; ++g) {
+          int mx0 = static_cast<int>(sr[g >> 1][(g & 1) * 16]);
+          int mx1 = static_cast<int>(sr[g >> 1][(g & 1) * 16 + 1]);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = (16 * g + e) >> 5, ee = (16 * g + e) & 31;
-            mx = max(mx, static_cast<int>(sr[c][ee]));
+          for (int e = 2; e < 16; e += 2) {
+            mx0 = max(mx0, static_cast<int>(sr[g >> 1][(g & 1) * 16 + e]));
+            mx1 = max(mx1, static_cast<int>(sr[g >> 1][(g & 1) * 16 + e + 1]));
           }
-          if (key < cand_hi) {
-            const float sk = skp[key / a.bk];
-            if (static_cast<float>(mx) * (cq * sk) >= thr) gbits |= 1u << g;
-          }
+          const int key = key0 + 16 * g;
+          if (key < cand_hi &&
+              static_cast<float>(max(mx0, mx1)) * cscale[key / a.bk] >= thr)
+            gbits |= 1u << g;
         }
         gbits = __reduce_or_sync(0xffffffffu, gbits);
         if (lane == 0 && gbits) {
-          const int g0 = (key0 - cand_lo) / 16;     // first group of this half-tile
-#pragma unroll
-          for (int g = 0; g < 8; ++g)
-            if ((gbits >> g) & 1u) atomicOr(&gflags[(g0 + g) >> 5], 1u << ((g0 + g) & 31));
+          const int g0 = (key0 - cand_lo) / 16;    // multiple of 4: one word holds all 4 bits
+          atomicOr(&gflags[g0 >> 5], gbits << (g0 & 31));
         }
       }
     }
-    (void)n_groups;
   }
   tc_fence_before();
   __syncthreads();

@@ -187,11 +187,20 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
       const int d = r;
       const uint32_t half = (d >> 6) * kHalfBytes;
       const uint32_t byte = (d & 63) * 2;
-      for (int rr = 0; rr < nrows; ++rr) {
-        const __nv_bfloat16 v =
-            *reinterpret_cast<const __nv_bfloat16*>(smem + half + sw128_offset(rr, byte));
-        acc += __bfloat162float(v);
+      auto qv = [&](int rr) {
+        return __bfloat162float(
+            *reinterpret_cast<const __nv_bfloat16*>(smem + half + sw128_offset(rr, byte)));
+      };
+      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;   // four independent chains
+      int rr = 0;
+      for (; rr + 4 <= nrows; rr += 4) {
+        p0 += qv(rr);
+        p1 += qv(rr + 1);
+        p2 += qv(rr + 2);
+        p3 += qv(rr + 3);
       }
+      for (; rr < nrows; ++rr) p0 += qv(rr);
+      acc = (p0 + p1) + (p2 + p3);
       const float qbar = (acc / static_cast<float>(nrows)) * a.scale;
       const __nv_bfloat16 hi = __float2bfloat16_rn(qbar);
       const __nv_bfloat16 lo = __float2bfloat16_rn(qbar - __bfloat162float(hi));
@@ -213,10 +222,14 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
 // ---------------------------------------------------------------------------
 // pooled-score scan: bitmask[bh][qb][word] over keys
 // ---------------------------------------------------------------------------
-constexpr int kScanThreads = 192;
+// One CTA: 128 query blocks (rows of the pooled-Q tile) x up to 16 key tiles.
+// Four TMEM accumulators of 128 columns let the MMA run three tiles ahead of
+// the epilogue; warps 2-9 each own one TMEM lane quadrant and 64 columns.
+constexpr int kScanThreads = 320;
 constexpr int kScanStages = 3;
+constexpr int kScanBufs = 4;
 constexpr int kScanTilesPerChunk = 16;
-constexpr uint32_t kScanSmemBytes = 1024u + 2u * kTileBytes + kScanStages * kTileBytes + 256u;
+constexpr uint32_t kScanSmemBytes = 1024u + 2u * kTileBytes + kScanStages * kTileBytes + 512u;
 
 struct ScanArgs {
   int B, Hq, Hkv, L, nqb, group;
@@ -255,31 +268,31 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
   uint8_t* bar_area = smem + 2 * kTileBytes + kScanStages * kTileBytes;
   const uint32_t b0 = smem_u32(bar_area);
   const uint32_t bar_a = b0;
-  auto bar_full = [&](int s) { return b0 + 8u * (1 + s); };
-  auto bar_empty = [&](int s) { return b0 + 8u * (1 + kScanStages + s); };
-  const uint32_t bar_sfull0 = b0 + 8u * (1 + 2 * kScanStages);
-  const uint32_t bar_sfree0 = bar_sfull0 + 16u;
-  const uint32_t bar_drain = bar_sfull0 + 32u;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 8 * (1 + 2 * kScanStages) + 40);
+  auto bar_full = [&](int st) { return b0 + 8u * (1 + st); };
+  auto bar_empty = [&](int st) { return b0 + 8u * (1 + kScanStages + st); };
+  auto bar_sfull = [&](int bb) { return b0 + 8u * (1 + 2 * kScanStages + bb); };
+  auto bar_sfree = [&](int bb) { return b0 + 8u * (1 + 2 * kScanStages + kScanBufs + bb); };
+  const uint32_t bar_drain = b0 + 8u * (1 + 2 * kScanStages + 2 * kScanBufs);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 256);
   volatile uint32_t* abort_flag = tmem_holder + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
     mbar_init(bar_a, 1);
-    for (int s = 0; s < kScanStages; ++s) {
-      mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
+    for (int st = 0; st < kScanStages; ++st) {
+      mbar_init(bar_full(st), 1);
+      mbar_init(bar_empty(st), 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_sfull0 + 8u * i, 1);
-      mbar_init(bar_sfree0 + 8u * i, 128);
+    for (int i = 0; i < kScanBufs; ++i) {
+      mbar_init(bar_sfull(i), 1);
+      mbar_init(bar_sfree(i), 256);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), 256);
+    tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -319,21 +332,23 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
     if (lane == 0) {
       bool ok = mbar_wait(bar_a, 0, wc);
       for (int t = 0; ok && t < T; ++t) {
-        const int st = t % kScanStages, bb = t & 1;
+        const int st = t % kScanStages, bb = t % kScanBufs;
         if (!(ok = mbar_wait(bar_full(st), (t / kScanStages) & 1, wc))) break;
-        if (t >= 2 && !(ok = mbar_wait(bar_sfree0 + 8u * bb, ((t - 2) >> 1) & 1, wc))) break;
+        if (t >= kScanBufs &&
+            !(ok = mbar_wait(bar_sfree(bb), ((t / kScanBufs) - 1) & 1, wc)))
+          break;
         tc_fence_after();
 #pragma unroll
         for (int part = 0; part < 2; ++part) {       // hi, then lo
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32u;
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32u;
             mma_bf16_ss(tmem + 128u * bb, smem_desc_sw128(s_a + part * kTileBytes + off, 16),
                         smem_desc_sw128(s_k(st) + off, 16), kIdescQK,
-                        (part > 0 || ks > 0) ? 1u : 0u);
+                        (part > 0 || kk > 0) ? 1u : 0u);
           }
         }
-        mma_commit(bar_sfull0 + 8u * bb);
+        mma_commit(bar_sfull(bb));
         mma_commit(bar_empty(st));
       }
       mma_commit(bar_drain);
@@ -342,6 +357,7 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
     __syncwarp();
   } else {
     const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;            // key columns [64*half, 64*half + 64)
     const int r = quad * 32 + lane;
     const int qb = qb_lo + r;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
@@ -350,30 +366,29 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
     const int cand_hi = row_valid ? max(0, (qb + 1) * 128 - a.local) : 0;   // ls of this block
     uint32_t* mrow = a.mask + ((long long)bh * a.nqb + (row_valid ? qb : 0)) * a.nwords;
     for (int t = 0; t < T; ++t) {
-      const int bb = t & 1;
-      if (!warp_wait(bar_sfull0 + 8u * bb, (t >> 1) & 1, wc)) break;
+      const int bb = t % kScanBufs;
+      if (!warp_wait(bar_sfull(bb), (t / kScanBufs) & 1, wc)) break;
       tc_fence_after();
-      uint32_t sr[4][32];
+      uint32_t sr[2][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + 128u * bb + 32u * c, sr[c]);
+      for (int c = 0; c < 2; ++c) tmem_ld32(tmem + lane_off + 128u * bb + 64u * half + 32u * c, sr[c]);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar_sfree0 + 8u * bb);
-      const int key0 = (t_lo + t) * 128;
-      // candidate keys of this row inside the tile: [lo, hi)
+      mbar_arrive(bar_sfree(bb));
+      const int key0 = (t_lo + t) * 128 + 64 * half;
+      // candidate keys of this row inside these 64 columns: [lo, hi)
       const int lo = max(a.sink - key0, 0);
-      const int hi = min(cand_hi - key0, 128);
-      uint4 wv;
+      const int hi = min(cand_hi - key0, 64);
+      uint2 wv;
       uint32_t* w = &wv.x;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         uint32_t bits = 0;
 #pragma unroll
         for (int e = 0; e < 32; ++e) {
           const float s = __uint_as_float(sr[c][e]);
           bits |= ((xb - s) <= a.theta ? 1u : 0u) << e;
         }
-        // keep only the candidate columns [lo, hi) of this word
         const int wlo = c * 32, whi = c * 32 + 32;
         const int l0 = max(lo, wlo) - wlo, l1 = min(hi, whi) - wlo;
         uint32_t range = 0;
@@ -381,14 +396,14 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
         w[c] = bits & range;
       }
       if (row_valid && key0 < cand_hi) {
-        *reinterpret_cast<uint4*>(mrow + key0 / 32) = wv;
+        *reinterpret_cast<uint2*>(mrow + key0 / 32) = wv;
       }
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
@@ -462,6 +477,90 @@ compact_kernel(const CompactArgs a) {
       if (wj == 0u) continue;                         // warp-uniform
       const int oj = __shfl_sync(0xffffffffu, excl, j);
       if ((wj >> lane) & 1u) out[base + oj + __popc(wj & lt)] = 32 * (w0 + j) + lane;
+    }
+    base += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// two heads' bitmasks -> one ascending union list with membership tags
+// ---------------------------------------------------------------------------
+// For the paired attention kernel (two q heads of one GQA group share every
+// K/V tile): entry = index | (in head 2p) << 30 | (in head 2p+1) << 31.
+struct PairCompactArgs {
+  int nqb, heads_q, sink, local, unit;
+  const uint32_t* mask;     // [B*Hq*nqb][nwords]
+  int nwords;
+  uint32_t* lists;          // [B*Hq/2][per_head] tagged entries
+  long long list_per_head;
+  long long cap_a;
+  int* counts;              // [B*Hq/2*nqb]
+};
+
+__global__ void __launch_bounds__(kCompactThreads)
+pair_compact_kernel(const PairCompactArgs a) {
+  const int row = blockIdx.x;                       // (b, pair, qb)
+  const int pair = row / a.nqb, qb = row - (row / a.nqb) * a.nqb;
+  const int b = pair / (a.heads_q / 2), pp = pair - b * (a.heads_q / 2);
+  const long long rowA = ((long long)b * a.heads_q + 2 * pp) * a.nqb + qb;
+  const long long rowB = rowA + a.nqb;
+  const int ls = max(0, (qb + 1) * 128 - a.local);
+  const int bit_lo = a.sink / a.unit;
+  const int bit_hi = max(a.sink, ls) / a.unit;
+  const int w_lo = bit_lo / 32;
+  const int w_hi = bit_hi > bit_lo ? (bit_hi + 31) / 32 : w_lo;
+  const int n = w_hi - w_lo;
+  const uint32_t* mA = a.mask + rowA * a.nwords;
+  const uint32_t* mB = a.mask + rowB * a.nwords;
+  uint32_t* out = a.lists + (long long)pair * a.list_per_head + cap_prefix(qb, 128, a.cap_a) / a.unit;
+
+  __shared__ int warp_cnt[kCompactThreads / 32];
+  __shared__ int warp_base[kCompactThreads / 32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nw = kCompactThreads / 32;
+  const int seg = (((n + nw - 1) / nw) + 31) & ~31;
+  const int s_lo = w_lo + warp * seg;
+  const int s_hi = min(s_lo + seg, w_hi);
+  int cnt = 0;
+  for (int w = s_lo + lane; w < s_hi; w += 32) cnt += __popc(mA[w] | mB[w]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (lane == 0) warp_cnt[warp] = cnt;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int i = 0; i < nw; ++i) {
+      warp_base[i] = run;
+      run += warp_cnt[i];
+    }
+    a.counts[row] = run;
+  }
+  __syncthreads();
+  int base = warp_base[warp];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int w0 = s_lo; w0 < s_hi; w0 += 32) {
+    const bool in = w0 + lane < s_hi;
+    const uint32_t wa = in ? mA[w0 + lane] : 0u;
+    const uint32_t wb = in ? mB[w0 + lane] : 0u;
+    const uint32_t word = wa | wb;
+    const int pc = __popc(word);
+    int incl = pc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    const int excl = incl - pc;
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t wj = __shfl_sync(0xffffffffu, word, j);
+      if (wj == 0u) continue;                         // warp-uniform
+      const uint32_t aj = __shfl_sync(0xffffffffu, wa, j);
+      const uint32_t bj = __shfl_sync(0xffffffffu, wb, j);
+      const int oj = __shfl_sync(0xffffffffu, excl, j);
+      if ((wj >> lane) & 1u) {
+        const uint32_t tag = (((aj >> lane) & 1u) << 30) | (((bj >> lane) & 1u) << 31);
+        out[base + oj + __popc(wj & lt)] = static_cast<uint32_t>(32 * (w0 + j) + lane) | tag;
+      }
     }
     base += __shfl_sync(0xffffffffu, incl, 31);
   }
