@@ -113,18 +113,18 @@ class ClockSampler:
 def _kernel_source_hash() -> str:
     import hashlib
     h = hashlib.sha256()
-    for name in ("attn.cuh", "ptx.cuh"):
+    for name in ("attn.cuh", "attn_pair.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "block_sparse_long_sm_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
 
 
-def _recorded_traffic(workload: str):
+def _recorded_traffic(workload: str, kernel: str):
     """DRAM bytes per launch of the attention kernel from the committed ncu
     record, only if the kernel source is the one the counters were taken on."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
-            rec = json.load(f)["sparse_attn_kernel"]
+            rec = json.load(f)[kernel]
     except Exception:
         return None
     if rec.get("source_sha256") != _kernel_source_hash() or rec.get("workload") != workload:
@@ -311,10 +311,14 @@ def main():
             "plan_ms": statistics.median(plan_ms), "attn_ms": statistics.median(attn_ms),
             "kept_fraction": stats.kept_pairs / stats.dense_pairs,
             "kept_flops_per_layer": flops_step,
-            "roofline": {"bound": "tensor", "kernel": "sparse_attn_kernel",
+            "roofline": {"bound": "tensor",
+                         "kernel": "sparse_attn_pair_kernel" if (w.heads_q // w.heads_kv) % 2 == 0
+                                   else "sparse_attn_kernel",
                          "achieved": achieved, "peak": peaks["bf16_sus"], "unit": "TFLOP/s",
                          "frac": achieved / peaks["bf16_sus"],
-                         "traffic": _recorded_traffic(w.name),
+                         "traffic": _recorded_traffic(
+                             w.name, "sparse_attn_pair_kernel" if (w.heads_q // w.heads_kv) % 2 == 0
+                             else "sparse_attn_kernel"),
                          "peak_source": f"{peaks['src']} bf16 dense, sustained (kernel timed inside a long loop)"},
             "clocks": clk.summary(),
             "gpu_launches": launches,

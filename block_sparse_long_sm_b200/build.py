@@ -1,14 +1,17 @@
 """Build the in-tree CUDA library ``lib/libspa.so`` for sm_100a with nvcc.
 
-Usage: ``python -m block_sparse_long_sm_b200.build`` (or ``build()`` from
-Python).  The build is incremental: it is skipped when the library is newer
-than every source under ``csrc/`` and ``include/``.
+Usage: ``python -m block_sparse_long_sm_b200.build [--force]`` (or
+``build()`` from Python).  The build is incremental: it is skipped when the
+library is newer than every source under ``csrc/`` and ``include/``.  Extra
+nvcc flags (for example ``-DSPA_EXP2_POLY_EVERY=4``) can be passed through
+the ``SPA_NVCC_EXTRA`` environment variable together with ``--force``.
 """
 
 from __future__ import annotations
 
 import glob
 import os
+import shlex
 import shutil
 import subprocess
 import sys
@@ -49,6 +52,7 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         return LIB
     os.makedirs(LIBDIR, exist_ok=True)
     tmp = LIB + ".tmp"
+    extra = list(extra) + shlex.split(os.environ.get("SPA_NVCC_EXTRA", ""))
     cmd = [_nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared",
            "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
            "-I", os.path.join(ROOT, "include"), "-o", tmp, *_sources(), *extra]

@@ -89,26 +89,30 @@ __global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
 // ---------------------------------------------------------------------------
 // fused sink-local statistics + block scan
 // ---------------------------------------------------------------------------
-// Tiles are 128 keys (M = 128 rows, N = 128, K = 128 int8 in four MMAs) so
-// that four TMEM accumulators (128 columns each) let the tensor core run up
-// to three tiles ahead of the epilogue.  Warps 2-9 form the epilogue: warp w
-// reads TMEM lanes 32*(w%4).. and columns [64*h, 64*h+64) of each tile,
-// h = (w-2)/4.  The per-key-block scales of the kv head are staged in shared
-// memory once per CTA.
+// One CTA = (b, kv head, query block, up to four q heads of that kv head's
+// group): the q heads share every int8 K tile, so each 64-key tile fetched
+// from L2 feeds up to four MMAs (M = 128 rows, N = 64, K = 128 in four
+// K = 32 steps).  TMEM: two accumulator sets x four heads x 64 columns.  The
+// epilogue (warps 2-9) gives each thread one row of two heads, all 64
+// columns of every tile, so the sink-local statistics need no cross-thread
+// merge.  Candidate tiles are read from TMEM as packed 16-bit pairs (the dots
+// fit: |dot| <= 7*7*128) and reduced with max.s16x2.
 constexpr int kSaleThreads = 320;            // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
-constexpr int kSaleStages = 4;
-constexpr int kSaleBufs = 4;                 // TMEM accumulators of 128 columns
+constexpr int kSaleStages = 8;
+constexpr int kSaleKeys = 64;                // keys per K tile
+constexpr int kSaleHeads = 4;                // q heads per CTA
 constexpr uint32_t kQ8Bytes = 128u * 128u;   // 128 rows x 128 int8
-constexpr uint32_t kK8Bytes = 128u * 128u;   // 128 keys x 128 int8
+constexpr uint32_t kK8Bytes = kSaleKeys * 128u;
 constexpr int kMaxGroupWords = 512;          // candidate 16-key groups / 32 (L <= 262144)
 constexpr int kMaxScales = 16384;            // key blocks per head (L / bk <= 16384)
-constexpr uint32_t kSaleSmemBytes = 1024u + kQ8Bytes + kSaleStages * kK8Bytes + 1024u +
-                                    kMaxGroupWords * 4u + 128u * 16u + kMaxScales * 4u;
-constexpr uint32_t kIdescI8N128 = make_idesc(2, 1, 128, 128, 0, 0);
+constexpr uint32_t kSaleSmemBytes = 1024u + kSaleHeads * kQ8Bytes + kSaleStages * kK8Bytes +
+                                    1024u + kSaleHeads * kMaxGroupWords * 4u + kMaxScales * 4u;
+constexpr uint32_t kIdescI8N64 = make_idesc(2, 1, 128, 64, 0, 0);
 
 struct SaleArgs {
   int B, Hq, Hkv, L, nqb, group;
   int sink, local, bk, nkb;
+  int chunks;               // ceil(group / kSaleHeads)
   float scale, tau;
   const float* sq;          // [B*Hq][nqb]
   const float* sk;          // [B*Hkv][nkb]
@@ -125,42 +129,44 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t s_q = s_base;
-  auto s_k = [&](int st) { return s_base + kQ8Bytes + st * kK8Bytes; };
-  uint8_t* bar_area = smem + kQ8Bytes + kSaleStages * kK8Bytes;
+  const uint32_t s_q = s_base;                                   // [head][128 x 128 int8]
+  auto s_k = [&](int st) { return s_base + kSaleHeads * kQ8Bytes + st * kK8Bytes; };
+  uint8_t* bar_area = smem + kSaleHeads * kQ8Bytes + kSaleStages * kK8Bytes;
   const uint32_t b0 = smem_u32(bar_area);
   const uint32_t bar_q = b0;
   auto bar_full = [&](int st) { return b0 + 8u * (1 + st); };
   auto bar_empty = [&](int st) { return b0 + 8u * (1 + kSaleStages + st); };
-  auto bar_sfull = [&](int bb) { return b0 + 8u * (1 + 2 * kSaleStages + bb); };
-  auto bar_sfree = [&](int bb) { return b0 + 8u * (1 + 2 * kSaleStages + kSaleBufs + bb); };
-  const uint32_t bar_drain = b0 + 8u * (1 + 2 * kSaleStages + 2 * kSaleBufs);
-  const uint32_t bar_stat = bar_drain + 8u;       // both column halves of every row posted
+  auto bar_afull = [&](int bb) { return b0 + 8u * (1 + 2 * kSaleStages + bb); };
+  auto bar_afree = [&](int bb) { return b0 + 8u * (3 + 2 * kSaleStages + bb); };
+  const uint32_t bar_drain = b0 + 8u * (5 + 2 * kSaleStages);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 512);
   volatile uint32_t* abort_flag = tmem_holder + 1;
-  uint32_t* gflags = reinterpret_cast<uint32_t*>(bar_area + 1024);    // candidate group flags
-  float* part = reinterpret_cast<float*>(gflags + kMaxGroupWords);    // [128][4]: m,l of 2 halves
-  float* cscale = part + 128 * 4;                                     // sq*sk*scale per key block
+  uint32_t* gflags = reinterpret_cast<uint32_t*>(bar_area + 1024);       // [head][words]
+  float* kscale = reinterpret_cast<float*>(gflags + kSaleHeads * kMaxGroupWords);  // sk*scale
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int x = blockIdx.x;
-  const int bh = x / a.nqb, qb = x - (x / a.nqb) * a.nqb;
-  const int b = bh / a.Hq, h = bh - b * a.Hq;
-  const int bkv = b * a.Hkv + h / a.group;
+  int x = blockIdx.x;
+  const int chunk = x % a.chunks;
+  x /= a.chunks;
+  const int qb = x % a.nqb;
+  const int bkv = x / a.nqb;                      // b * Hkv + kv head
+  const int b = bkv / a.Hkv, kvh = bkv - b * a.Hkv;
+  const int h0 = kvh * a.group + chunk * kSaleHeads;
+  const int nh = min(kSaleHeads, a.group - chunk * kSaleHeads);
   const int row0 = qb * 128;
   const int le = min(row0 + 128, a.L);
   const int ls = max(0, row0 + 128 - a.local);
   const int sink_end = min(a.sink, ls);
-  const int n_sink_t = (sink_end + 127) / 128;
-  const int n_loc_t = (le - ls + 127) / 128;
+  const int n_sink_t = (sink_end + kSaleKeys - 1) / kSaleKeys;
+  const int n_loc_t = (le - ls + kSaleKeys - 1) / kSaleKeys;
   const int cand_lo = a.sink, cand_hi = max(a.sink, ls);
-  const int n_cand_t = (cand_hi - cand_lo + 127) / 128;
+  const int n_cand_t = (cand_hi - cand_lo + kSaleKeys - 1) / kSaleKeys;
   const int n_stat_t = n_sink_t + n_loc_t;
   const int T = n_stat_t + n_cand_t;
   auto tile_key0 = [&](int t) {
-    if (t < n_sink_t) return t * 128;
-    if (t < n_stat_t) return ls + (t - n_sink_t) * 128;
-    return cand_lo + (t - n_stat_t) * 128;
+    if (t < n_sink_t) return t * kSaleKeys;
+    if (t < n_stat_t) return ls + (t - n_sink_t) * kSaleKeys;
+    return cand_lo + (t - n_stat_t) * kSaleKeys;
   };
 
   if (threadIdx.x == 0) {
@@ -169,21 +175,19 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
       mbar_init(bar_full(st), 1);
       mbar_init(bar_empty(st), 1);
     }
-    for (int i = 0; i < kSaleBufs; ++i) {
-      mbar_init(bar_sfull(i), 1);
-      mbar_init(bar_sfree(i), 256);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar_afull(i), 1);
+      mbar_init(bar_afree(i), 256);
     }
     mbar_init(bar_drain, 1);
-    mbar_init(bar_stat, 256);
     *abort_flag = 0u;
     fence_barrier_init();
   }
-  for (int i = threadIdx.x; i < kMaxGroupWords; i += blockDim.x) gflags[i] = 0u;
+  for (int i = threadIdx.x; i < kSaleHeads * kMaxGroupWords; i += blockDim.x) gflags[i] = 0u;
   {
-    const float cq = a.sq[(long long)bh * a.nqb + qb] * a.scale;
     const int nkb_used = min(a.nkb, (le + a.bk - 1) / a.bk);
     const float* skp = a.sk + (long long)bkv * a.nkb;
-    for (int i = threadIdx.x; i < nkb_used; i += blockDim.x) cscale[i] = cq * skp[i];
+    for (int i = threadIdx.x; i < nkb_used; i += blockDim.x) kscale[i] = skp[i] * a.scale;
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), 512);
@@ -197,8 +201,9 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
 
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, kQ8Bytes);
-      tma_load_2d(s_q, &tm_q8, bar_q, 0, bh * a.L + row0);
+      mbar_arrive_expect_tx(bar_q, nh * kQ8Bytes);
+      for (int j = 0; j < nh; ++j)
+        tma_load_2d(s_q + j * kQ8Bytes, &tm_q8, bar_q, 0, (b * a.Hq + h0 + j) * a.L + row0);
       int issued = 0;
       for (int t = 0; t < T; ++t) {
         const int st = t % kSaleStages;
@@ -218,18 +223,19 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
     if (lane == 0) {
       bool ok = mbar_wait(bar_q, 0, wc);
       for (int t = 0; ok && t < T; ++t) {
-        const int st = t % kSaleStages, bb = t % kSaleBufs;
+        const int st = t % kSaleStages, bb = t & 1;
         if (!(ok = mbar_wait(bar_full(st), (t / kSaleStages) & 1, wc))) break;
-        if (t >= kSaleBufs &&
-            !(ok = mbar_wait(bar_sfree(bb), ((t / kSaleBufs) - 1) & 1, wc)))
-          break;
+        if (t >= 2 && !(ok = mbar_wait(bar_afree(bb), ((t >> 1) - 1) & 1, wc))) break;
         tc_fence_after();
+        for (int j = 0; j < nh; ++j) {
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          mma_i8_ss(tmem + 128u * bb, smem_desc_sw128(s_q + kk * 32u, 16),
-                    smem_desc_sw128(s_k(st) + kk * 32u, 16), kIdescI8N128, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            mma_i8_ss(tmem + 64u * (bb * kSaleHeads + j),
+                      smem_desc_sw128(s_q + j * kQ8Bytes + kk * 32u, 16),
+                      smem_desc_sw128(s_k(st) + kk * 32u, 16), kIdescI8N64, kk > 0 ? 1u : 0u);
+          }
         }
-        mma_commit(bar_sfull(bb));
+        mma_commit(bar_afull(bb));
         mma_commit(bar_empty(st));
       }
       mma_commit(bar_drain);
@@ -238,105 +244,110 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
     __syncwarp();
   } else {
     const int quad = warp & 3;               // TMEM lane quadrant
-    const int half = (warp - 2) >> 2;        // columns [64*half, 64*half + 64)
+    const int hsel = (warp - 2) >> 2;        // heads hsel and hsel + 2
     const int r = quad * 32 + lane;
     const int row = row0 + r;
     const bool row_valid = row < a.L;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    float m = -INFINITY, l = 0.f, thr = INFINITY;
+    float cq[2], m[2], l[2], thr[2];
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const int j = hsel + 2 * u;
+      cq[u] = j < nh ? a.sq[((long long)b * a.Hq + h0 + j) * a.nqb + qb] : 0.f;
+      m[u] = -INFINITY;
+      l[u] = 0.f;
+      thr[u] = INFINITY;
+    }
     for (int t = 0; t < T; ++t) {
-      const int bb = t % kSaleBufs;
-      if (!warp_wait(bar_sfull(bb), (t / kSaleBufs) & 1, wc)) break;
+      const int bb = t & 1;
+      if (!warp_wait(bar_afull(bb), (t >> 1) & 1, wc)) break;
       tc_fence_after();
-      uint32_t sr[2][32];
+      const int key0 = tile_key0(t);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) tmem_ld32(tmem + lane_off + 128u * bb + 64u * half + 32u * c, sr[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar_sfree(bb));
-      const int key0 = tile_key0(t) + 64 * half;
-      if (t < n_stat_t) {
-        // S~ over the causal sink-local keys of this row
-        int limit = (t < n_sink_t) ? sink_end - key0 : min(le - key0, row - key0 + 1);
-        limit = max(0, min(limit, 64));
-        float tm = -INFINITY;
+      for (int u = 0; u < 2; ++u) {
+        const int j = hsel + 2 * u;
+        if (j >= nh) continue;                         // warp-uniform
+        const uint32_t taddr = tmem + lane_off + 64u * (bb * kSaleHeads + j);
+        if (t < n_stat_t) {
+          uint32_t sr[2][32];
+          tmem_ld32(taddr, sr[0]);
+          tmem_ld32(taddr + 32u, sr[1]);
+          tmem_ld_wait();
+          // S~ over the causal sink-local keys of this row
+          int limit = (t < n_sink_t) ? sink_end - key0 : min(le - key0, row - key0 + 1);
+          limit = max(0, min(limit, kSaleKeys));
+          float tm = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+          for (int c = 0; c < 2; ++c) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int col = c * 32 + e;
-            const float v = col < limit
-                                ? static_cast<float>(static_cast<int>(sr[c][e])) *
-                                      cscale[min(key0 + col, a.L - 1) / a.bk]
-                                : -INFINITY;
-            sr[c][e] = __float_as_uint(v);
-            tm = fmaxf(tm, v);
+            for (int e = 0; e < 32; ++e) {
+              const int col = c * 32 + e;
+              const float v = col < limit
+                                  ? static_cast<float>(static_cast<int>(sr[c][e])) *
+                                        (cq[u] * kscale[min(key0 + col, a.L - 1) / a.bk])
+                                  : -INFINITY;
+              sr[c][e] = __float_as_uint(v);
+              tm = fmaxf(tm, v);
+            }
           }
-        }
-        if (tm > -INFINITY) {
-          const float mn = fmaxf(m, tm);
-          float acc = 0.f;
+          if (tm > -INFINITY) {
+            const float mn = fmaxf(m[u], tm);
+            float acc = 0.f;
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+            for (int c = 0; c < 2; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e) acc += __expf(__uint_as_float(sr[c][e]) - mn);
-          l = l * __expf(m - mn) + acc;
-          m = mn;
-        }
-        if (t == n_stat_t - 1) {
-          // merge the two column halves of each row, then t_i = em + ln(tau el)
-          part[r * 4 + half * 2 + 0] = m;
-          part[r * 4 + half * 2 + 1] = l;
-          mbar_arrive(bar_stat);
-          if (!warp_wait(bar_stat, 0, wc)) break;
-          const float m0 = part[r * 4 + 0], l0 = part[r * 4 + 1];
-          const float m1 = part[r * 4 + 2], l1 = part[r * 4 + 3];
-          const float em = fmaxf(m0, m1);
-          const float el = (m0 > -INFINITY ? l0 * expf(m0 - em) : 0.f) +
-                           (m1 > -INFINITY ? l1 * expf(m1 - em) : 0.f);
-          thr = row_valid ? em + logf(a.tau * el) : INFINITY;
-        }
-      } else {
-        // candidate tile: one flag per 16-key group (groups never straddle ls)
-        uint32_t gbits = 0;
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          int mx0 = static_cast<int>(sr[g >> 1][(g & 1) * 16]);
-          int mx1 = static_cast<int>(sr[g >> 1][(g & 1) * 16 + 1]);
-#pragma unroll
-          for (int e = 2; e < 16; e += 2) {
-            mx0 = max(mx0, static_cast<int>(sr[g >> 1][(g & 1) * 16 + e]));
-            mx1 = max(mx1, static_cast<int>(sr[g >> 1][(g & 1) * 16 + e + 1]));
+              for (int e = 0; e < 32; ++e) acc += __expf(__uint_as_float(sr[c][e]) - mn);
+            l[u] = l[u] * __expf(m[u] - mn) + acc;
+            m[u] = mn;
           }
-          const int key = key0 + 16 * g;
-          if (key < cand_hi &&
-              static_cast<float>(max(mx0, mx1)) * cscale[key / a.bk] >= thr)
-            gbits |= 1u << g;
-        }
-        gbits = __reduce_or_sync(0xffffffffu, gbits);
-        if (lane == 0 && gbits) {
-          const int g0 = (key0 - cand_lo) / 16;    // multiple of 4: one word holds all 4 bits
-          atomicOr(&gflags[g0 >> 5], gbits << (g0 & 31));
+          if (t == n_stat_t - 1)
+            thr[u] = row_valid ? m[u] + logf(a.tau * l[u]) : INFINITY;   // t_i = em + ln(tau el)
+        } else {
+          uint32_t pk[32];
+          tmem_ld32_pack16(taddr, pk);
+          tmem_ld_wait();
+          uint32_t gbits = 0;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {               // 16 keys = 8 packed registers
+            const uint32_t* q = pk + 8 * g;
+            const uint32_t m01 = max_s16x2(max_s16x2(q[0], q[1]), max_s16x2(q[2], q[3]));
+            const uint32_t m23 = max_s16x2(max_s16x2(q[4], q[5]), max_s16x2(q[6], q[7]));
+            const uint32_t mm = max_s16x2(m01, m23);
+            const int mx = max(static_cast<int>(static_cast<int16_t>(mm & 0xffffu)),
+                               static_cast<int>(mm) >> 16);
+            const int key = key0 + 16 * g;
+            if (key < cand_hi && static_cast<float>(mx) * (cq[u] * kscale[key / a.bk]) >= thr[u])
+              gbits |= 1u << g;
+          }
+          gbits = __reduce_or_sync(0xffffffffu, gbits);
+          if (lane == 0 && gbits) {
+            const int g0 = (key0 - cand_lo) / 16;    // multiple of 4: one word holds all 4 bits
+            atomicOr(&gflags[j * kMaxGroupWords + (g0 >> 5)], gbits << (g0 & 31));
+          }
         }
       }
+      tc_fence_before();
+      mbar_arrive(bar_afree(bb));
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // key-block flags -> global bitmask row (every word of the row is written)
+  // key-block flags -> global bitmask rows (every word of every row is written)
   if (!*abort_flag) {
     const int gpb = a.bk / 16;                     // groups per key block
     const int kb_lo = cand_lo / a.bk;
-    uint32_t* mrow = a.mask + (long long)x * a.nwords;
-    for (int w = threadIdx.x; w < a.nwords; w += blockDim.x) {
+    for (int idx = threadIdx.x; idx < nh * a.nwords; idx += blockDim.x) {
+      const int j = idx / a.nwords, w = idx - j * a.nwords;
+      uint32_t* mrow = a.mask + (((long long)b * a.Hq + h0 + j) * a.nqb + qb) * a.nwords;
+      const uint32_t* gf = gflags + j * kMaxGroupWords;
       uint32_t word = 0;
       for (int bit = 0; bit < 32; ++bit) {
         const int kb = w * 32 + bit;
         if (kb < kb_lo || kb * a.bk >= cand_hi) continue;
         const int g0 = (kb - kb_lo) * gpb;
         bool any = false;
-        for (int g = g0; g < g0 + gpb; ++g) any |= (gflags[g >> 5] >> (g & 31)) & 1u;
+        for (int g = g0; g < g0 + gpb; ++g) any |= (gf[g >> 5] >> (g & 31)) & 1u;
         word |= (any ? 1u : 0u) << bit;
       }
       mrow[w] = word;

@@ -417,6 +417,7 @@ struct CompactArgs {
   int L;
   int sink, local;
   int unit;                 // 1: bits are keys; bk: bits are key blocks
+  int step;                 // query blocks per selection group (>= 1)
   const uint32_t* mask;     // [rows][nwords]
   int nwords;
   int* lists;
@@ -435,8 +436,23 @@ compact_kernel(const CompactArgs a) {
   const int w_lo = bit_lo / 32;
   const int w_hi = bit_hi > bit_lo ? (bit_hi + 31) / 32 : w_lo;
   const int n = w_hi - w_lo;
-  const uint32_t* m = a.mask + (long long)row * a.nwords;
   int* out = a.lists + (long long)bh * a.list_per_head + cap_prefix(qb, 128, a.cap_a) / a.unit;
+  // Selection groups (step > 1): a word is the OR of the group's rows, each
+  // read only inside its own candidate range (the rest of a row is never
+  // written) -- the result is then cut to this block's range by [w_lo, w_hi).
+  const int g0 = (qb / a.step) * a.step;
+  const int g1 = min(g0 + a.step, a.nqb);
+  const uint32_t* mrow0 = a.mask + ((long long)row - qb) * a.nwords;   // block 0 of this head
+  auto word_at = [&](int w) -> uint32_t {
+    if (a.step == 1) return mrow0[(long long)qb * a.nwords + w];
+    uint32_t v = 0;
+    for (int b2 = g0; b2 < g1; ++b2) {
+      const int ls2 = max(0, (b2 + 1) * 128 - a.local);
+      const int hi2 = max(a.sink, ls2) / a.unit;
+      if (w < (hi2 + 31) / 32) v |= mrow0[(long long)b2 * a.nwords + w];
+    }
+    return v;
+  };
 
   __shared__ int warp_cnt[kCompactThreads / 32];
   __shared__ int warp_base[kCompactThreads / 32];
@@ -446,7 +462,7 @@ compact_kernel(const CompactArgs a) {
   const int s_lo = w_lo + warp * seg;
   const int s_hi = min(s_lo + seg, w_hi);
   int cnt = 0;
-  for (int w = s_lo + lane; w < s_hi; w += 32) cnt += __popc(m[w]);
+  for (int w = s_lo + lane; w < s_hi; w += 32) cnt += __popc(word_at(w));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
   if (lane == 0) warp_cnt[warp] = cnt;
@@ -463,7 +479,7 @@ compact_kernel(const CompactArgs a) {
   int base = warp_base[warp];
   const uint32_t lt = (1u << lane) - 1u;
   for (int w0 = s_lo; w0 < s_hi; w0 += 32) {
-    const uint32_t word = (w0 + lane < s_hi) ? m[w0 + lane] : 0u;
+    const uint32_t word = (w0 + lane < s_hi) ? word_at(w0 + lane) : 0u;
     const int pc = __popc(word);
     int incl = pc;
 #pragma unroll
@@ -488,7 +504,7 @@ compact_kernel(const CompactArgs a) {
 // For the paired attention kernel (two q heads of one GQA group share every
 // K/V tile): entry = index | (in head 2p) << 30 | (in head 2p+1) << 31.
 struct PairCompactArgs {
-  int nqb, heads_q, sink, local, unit;
+  int nqb, heads_q, sink, local, unit, step;
   const uint32_t* mask;     // [B*Hq*nqb][nwords]
   int nwords;
   uint32_t* lists;          // [B*Hq/2][per_head] tagged entries
@@ -510,8 +526,27 @@ pair_compact_kernel(const PairCompactArgs a) {
   const int w_lo = bit_lo / 32;
   const int w_hi = bit_hi > bit_lo ? (bit_hi + 31) / 32 : w_lo;
   const int n = w_hi - w_lo;
-  const uint32_t* mA = a.mask + rowA * a.nwords;
-  const uint32_t* mB = a.mask + rowB * a.nwords;
+  const int g0 = (qb / a.step) * a.step;
+  const int g1 = min(g0 + a.step, a.nqb);
+  const uint32_t* mA0 = a.mask + (rowA - qb) * a.nwords;     // block 0 of head A
+  const uint32_t* mB0 = a.mask + (rowB - qb) * a.nwords;
+  auto words_at = [&](int w, uint32_t& wa, uint32_t& wb) {
+    if (a.step == 1) {
+      wa = mA0[(long long)qb * a.nwords + w];
+      wb = mB0[(long long)qb * a.nwords + w];
+      return;
+    }
+    wa = 0u;
+    wb = 0u;
+    for (int b2 = g0; b2 < g1; ++b2) {
+      const int ls2 = max(0, (b2 + 1) * 128 - a.local);
+      const int hi2 = max(a.sink, ls2) / a.unit;
+      if (w < (hi2 + 31) / 32) {
+        wa |= mA0[(long long)b2 * a.nwords + w];
+        wb |= mB0[(long long)b2 * a.nwords + w];
+      }
+    }
+  };
   uint32_t* out = a.lists + (long long)pair * a.list_per_head + cap_prefix(qb, 128, a.cap_a) / a.unit;
 
   __shared__ int warp_cnt[kCompactThreads / 32];
@@ -522,7 +557,11 @@ pair_compact_kernel(const PairCompactArgs a) {
   const int s_lo = w_lo + warp * seg;
   const int s_hi = min(s_lo + seg, w_hi);
   int cnt = 0;
-  for (int w = s_lo + lane; w < s_hi; w += 32) cnt += __popc(mA[w] | mB[w]);
+  for (int w = s_lo + lane; w < s_hi; w += 32) {
+    uint32_t wa, wb;
+    words_at(w, wa, wb);
+    cnt += __popc(wa | wb);
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
   if (lane == 0) warp_cnt[warp] = cnt;
@@ -539,9 +578,8 @@ pair_compact_kernel(const PairCompactArgs a) {
   int base = warp_base[warp];
   const uint32_t lt = (1u << lane) - 1u;
   for (int w0 = s_lo; w0 < s_hi; w0 += 32) {
-    const bool in = w0 + lane < s_hi;
-    const uint32_t wa = in ? mA[w0 + lane] : 0u;
-    const uint32_t wb = in ? mB[w0 + lane] : 0u;
+    uint32_t wa = 0u, wb = 0u;
+    if (w0 + lane < s_hi) words_at(w0 + lane, wa, wb);
     const uint32_t word = wa | wb;
     const int pc = __popc(word);
     int incl = pc;

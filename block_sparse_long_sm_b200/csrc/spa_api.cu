@@ -11,6 +11,7 @@
 
 #include "../../include/spa.h"
 #include "attn.cuh"
+#include "attn_pair.cuh"
 #include "ptx.cuh"
 #include "sale.cuh"
 #include "select.cuh"
@@ -33,6 +34,8 @@ struct Layout {
   int nwords = 0;                   // bitmask words per block row
   size_t counts = 0, lists = 0, xbar = 0, qbar = 0, mask = 0;
   size_t kpart = 0, kmean = 0, q8 = 0, k8 = 0, sq = 0, sk = 0;
+  bool paired = false;              // two q heads per attention CTA (Hq / Hkv even)
+  size_t pair_counts = 0, pair_lists = 0;
   size_t total = 0;
 };
 
@@ -44,7 +47,7 @@ spa_status validate(const spa_params* p) {
   if (p->head_dim != 128) return SPA_ERR_UNSUPPORTED;
   if (p->causal != 1) return SPA_ERR_UNSUPPORTED;
   if (p->block_q != 128) return SPA_ERR_UNSUPPORTED;
-  if (p->step != 1) return SPA_ERR_UNSUPPORTED;
+  if (p->step < 1) return SPA_ERR_INVALID;
   if (p->sink < 0) return SPA_ERR_INVALID;
   if (p->local < p->block_q || p->local % p->block_q != 0) return SPA_ERR_INVALID;
   if (!(p->softmax_scale >= 0.f) || !std::isfinite(p->softmax_scale)) return SPA_ERR_INVALID;
@@ -113,6 +116,12 @@ Layout layout_of(const spa_params* p) {
   } else {
     lo.unit = 1;
     lo.counts = take(lo.nb * 4);
+  }
+  lo.paired = (lo.group % 2) == 0;
+  if (lo.paired && p->mode != SPA_MODE_DENSE) {
+    // union lists of head pairs for the paired attention kernel (opaque scratch)
+    lo.pair_counts = take((lo.nb / 2) * 4);
+    lo.pair_lists = take((size_t)(bh / 2) * lo.list_per_head * 4);
   }
   lo.total = off;
   lo.ok = true;
@@ -277,22 +286,32 @@ SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
     CUtensorMap tq8, tk8;
     if (!map_2d(&tq8, kI8, 1, ws + lo.q8, 128, BH * L, 128, 128, kSW128) ||
-        !map_2d(&tk8, kI8, 1, ws + lo.k8, 128, BKV * L, 128, 256, kSW128))
+        !map_2d(&tk8, kI8, 1, ws + lo.k8, 128, BKV * L, 128, kSaleKeys, kSW128))
       return SPA_ERR_CUDA;
+    const int chunks = (lo.group + kSaleHeads - 1) / kSaleHeads;
     SaleArgs sa{B, Hq, Hkv, L, lo.nqb, lo.group, p->sink, p->local, p->block_k, lo.nkb,
-                scale, p->tau, reinterpret_cast<const float*>(ws + lo.sq),
+                chunks, scale, p->tau, reinterpret_cast<const float*>(ws + lo.sq),
                 reinterpret_cast<const float*>(ws + lo.sk),
                 reinterpret_cast<uint32_t*>(ws + lo.mask), lo.nwords, err, wait_ns(p)};
     if (set_smem(sale_scan_kernel, kSaleSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
-    sale_scan_kernel<<<(unsigned)lo.nb, kSaleThreads, kSaleSmemBytes, stream>>>(tq8, tk8, sa);
+    sale_scan_kernel<<<(unsigned)(BKV * lo.nqb * chunks), kSaleThreads, kSaleSmemBytes,
+                       stream>>>(tq8, tk8, sa);
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   }
-  CompactArgs ca{(int)lo.nb, lo.nqb, L, p->sink, p->local, lo.unit,
+  CompactArgs ca{(int)lo.nb, lo.nqb, L, p->sink, p->local, lo.unit, p->step,
                  reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
                  reinterpret_cast<int*>(ws + lo.lists), lo.list_per_head, lo.cap_a,
                  reinterpret_cast<int*>(ws + lo.counts)};
   compact_kernel<<<(unsigned)lo.nb, kCompactThreads, 0, stream>>>(ca);
   if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
+  if (lo.paired) {
+    PairCompactArgs pc{lo.nqb, Hq, p->sink, p->local, lo.unit, p->step,
+                       reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
+                       reinterpret_cast<uint32_t*>(ws + lo.pair_lists), lo.list_per_head, lo.cap_a,
+                       reinterpret_cast<int*>(ws + lo.pair_counts)};
+    pair_compact_kernel<<<(unsigned)(lo.nb / 2), kCompactThreads, 0, stream>>>(pc);
+    if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
+  }
   return SPA_OK;
 }
 
@@ -327,14 +346,23 @@ SPA_API spa_status sparse_prefill_attn(const spa_params* p, const void* q, const
   aa.list_per_head = lo.list_per_head;
   aa.cap_a = lo.cap_a;
   aa.list_unit = lo.unit;
+  aa.pair_counts = reinterpret_cast<const int*>(ws + lo.pair_counts);
+  aa.pair_lists = reinterpret_cast<const uint32_t*>(ws + lo.pair_lists);
+  aa.pair_per_head = lo.list_per_head;
   aa.o = static_cast<__nv_bfloat16*>(o);
   aa.lse = lse;
   aa.err = reinterpret_cast<uint32_t*>(ws);
   aa.wait_ns = wait_ns(p);
   aa.debug = p->debug_flags;
-  if (set_smem(sparse_attn_kernel, kAttnSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
-  sparse_attn_kernel<<<(unsigned)lo.nb, kAttnThreads, kAttnSmemBytes, stream>>>(tq, tk, tkg, tv,
-                                                                               tvg, aa);
+  if (lo.paired) {
+    if (set_smem(sparse_attn_pair_kernel, kPairSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
+    sparse_attn_pair_kernel<<<(unsigned)(lo.nb / 2), kPairThreads, kPairSmemBytes, stream>>>(
+        tq, tk, tkg, tv, tvg, aa);
+  } else {
+    if (set_smem(sparse_attn_kernel, kAttnSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
+    sparse_attn_kernel<<<(unsigned)lo.nb, kAttnThreads, kAttnSmemBytes, stream>>>(tq, tk, tkg,
+                                                                                 tv, tvg, aa);
+  }
   if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   return SPA_OK;
 }
@@ -494,7 +522,7 @@ SPA_API spa_status sparse_prefill_plan_static(const spa_params* p, const void* q
                          stream>>>(tqbar, tk, sa);
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   }
-  CompactArgs ca{(int)lo.nb, lo.nqb, L, p->sink, p->local, 1,
+  CompactArgs ca{(int)lo.nb, lo.nqb, L, p->sink, p->local, 1, p->step,
                  reinterpret_cast<const uint32_t*>(ws + sl.mask), lo.nwords, lists,
                  lo.list_per_head, lo.cap_a, counts};
   compact_kernel<<<(unsigned)lo.nb, kCompactThreads, 0, stream>>>(ca);

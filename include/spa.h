@@ -74,7 +74,7 @@ extern "C" {
 typedef enum {
   SPA_OK = 0,
   SPA_ERR_INVALID = 1,      /* bad argument (null/misaligned pointer, bad size or value) */
-  SPA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head_dim != 128, causal == 0, step != 1, ...) */
+  SPA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (head_dim != 128, causal == 0, ...) */
   SPA_ERR_WORKSPACE = 3,    /* workspace smaller than sparse_prefill_workspace_bytes() */
   SPA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
   SPA_ERR_TIMEOUT = 5       /* a device-side bounded wait expired (reported by stats) */
@@ -97,7 +97,10 @@ typedef struct {
   int32_t block_k;        /* ANCHOR: 1 (key stripes); SALE: 16, 32, 64 or 128; DENSE: ignored */
   int32_t sink;           /* >= 0; SALE: multiple of block_k */
   int32_t local;          /* >= block_q, multiple of block_q */
-  int32_t step;           /* query blocks grouped per selection; must be 1 */
+  int32_t step;           /* >= 1: query blocks grouped per selection (AnchorAttention's
+                             step); a candidate kept by any block of a group of `step`
+                             consecutive blocks is kept by all of them, within each
+                             block's own candidate range.  1 = each block for itself */
   spa_mode mode;
   float theta;            /* ANCHOR threshold, scaled-logit units; +inf keeps all; NaN invalid */
   float tau;              /* SALE threshold on the relative score, 0 < tau <= 1 */

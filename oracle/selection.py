@@ -291,3 +291,29 @@ def sale_blocks_to_keys(kept_blocks: np.ndarray, bk: int) -> np.ndarray:
     if kept_blocks.size == 0:
         return np.zeros(0, dtype=np.int64)
     return (kept_blocks[:, None] * bk + np.arange(bk)[None, :]).reshape(-1)
+
+
+# ---------------------------------------------------------------------------
+# Query-block grouping (AnchorAttention's ``step``)
+# ---------------------------------------------------------------------------
+
+def step_union(selected_of_block, qb: int, *, step: int, nqb: int, cand_lo: int,
+               cand_hi: int) -> np.ndarray:
+    """Selection of block ``qb`` when query blocks are grouped ``step`` at a time.
+
+    AnchorAttention (Sec. 3.4; Appendix C, Algorithm 2 with the ``step``
+    parameter): the identification runs for groups of ``step`` consecutive
+    query blocks and a key selected by any block of the group is active for
+    every block of the group.  Reading taken here: the group of block b is
+    [floor(b / step) * step, ... + step) (clipped to the layer), the union is
+    taken over the blocks' own selections, and it is restricted to block b's
+    own candidate range [cand_lo, cand_hi) so that no key outside b's causal
+    candidates (or inside its always-kept sink/local windows) is added.
+    ``selected_of_block(b)`` returns block b's own selection (keys, or key-block
+    ids with a range given in the same units).
+    """
+    g0 = (qb // step) * step
+    parts = [np.asarray(selected_of_block(b), dtype=np.int64)
+             for b in range(g0, min(g0 + step, nqb))]
+    keys = np.unique(np.concatenate(parts)) if parts else np.zeros(0, dtype=np.int64)
+    return keys[(keys >= cand_lo) & (keys < cand_hi)]

@@ -38,13 +38,13 @@ class Run:
 
     def __init__(self, inputs: Inputs, *, mode: str, sink: int, local: int, theta: float = 5.0,
                  tau: float = 1e-3, block_k=None, do_attn: bool = True, lse: bool = True,
-                 dev=None):
+                 dev=None, step: int = 1):
         B, Hq, L, _ = inputs.q.shape
         Hkv = inputs.k.shape[1]
         self.B, self.Hq, self.Hkv, self.L = B, Hq, Hkv, L
         self.group = Hq // Hkv
         self.params = spa.make_params(B, Hq, Hkv, L, mode=mode, sink=sink, local=local,
-                                      theta=theta, tau=tau, block_k=block_k)
+                                      theta=theta, tau=tau, block_k=block_k, step=step)
         self.q, self.k, self.v = dev if dev is not None else (
             to_dev(inputs.q), to_dev(inputs.k), to_dev(inputs.v))
         nbytes = spa.sparse_prefill_workspace_bytes(self.params)
@@ -94,23 +94,39 @@ def check_list_shape(lst: np.ndarray, lo: int, hi: int):
 
 def compare_anchor_masks(run: Run, inputs: Inputs, heads: Sequence[Tuple[int, int]],
                          blocks_of=None, theta: float = None) -> Dict[str, int]:
-    """Selection parity for the given (b, h) heads; returns mismatch counts."""
+    """Selection parity for the given (b, h) heads; returns mismatch counts.
+
+    With step > 1 the oracle's selection of a block is the union over its
+    group (oracle.selection.step_union); a key may differ only if its decision
+    is a near-tie in some block of the group.
+    """
     p = run.params
     theta = p.theta if theta is None else theta
+    step = int(p.step)
     nqb = (run.L + 127) // 128
     total = dict(blocks=0, kept=0, mismatches=0, near_tie=0)
     for b, h in heads:
         qh = head_f64(inputs.q, b, h)
         kh = head_f64(inputs.k, b, h // run.group)
         blocks = list(range(nqb)) if blocks_of is None else list(blocks_of(b, h))
-        ora = osel.anchor_head(qh, kh, blocks, bq=128, sink=p.sink, local=p.local, theta=theta)
+        need = sorted({g for qb in blocks
+                       for g in range((qb // step) * step, min((qb // step) * step + step, nqb))})
+        ora = osel.anchor_head(qh, kh, need, bq=128, sink=p.sink, local=p.local, theta=theta)
         for qb in blocks:
             o = ora[qb]
+            kept = osel.step_union(lambda x: ora[x].kept, qb, step=step, nqb=nqb,
+                                   cand_lo=o.cand[0] if o.cand.size else p.sink,
+                                   cand_hi=(o.cand[-1] + 1) if o.cand.size else p.sink)
             g = run.block_list(b, h, qb)
             check_list_shape(g, o.cand[0] if o.cand.size else p.sink, (o.cand[-1] + 1) if o.cand.size else p.sink)
-            diff = np.setxor1d(g, o.kept)
+            diff = np.setxor1d(g, kept)
             if diff.size:
-                m = o.margin[diff - p.sink]
+                g0 = (qb // step) * step
+                m = np.full(diff.shape, np.inf)
+                for b2 in range(g0, min(g0 + step, nqb)):
+                    c2 = ora[b2].cand
+                    inside = (diff >= p.sink) & (diff < p.sink + c2.size)
+                    m[inside] = np.minimum(m[inside], np.abs(ora[b2].margin[diff[inside] - p.sink]))
                 bad = np.abs(m) >= MASK_MARGIN
                 assert not bad.any(), (
                     f"mask mismatch b={b} h={h} qb={qb}: keys {diff[bad][:8]} margins {m[bad][:8]}")

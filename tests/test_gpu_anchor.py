@@ -117,3 +117,44 @@ def test_stats_match_oracle_counts():
     assert run.stats.kept_candidates == int(run.counts.sum())
     assert run.stats.dense_pairs == L * (L + 1) // 2
     assert run.stats.query_blocks == nqb
+
+
+@pytest.mark.parametrize("hq,hkv,mode", [(3, 1, "anchor"), (6, 2, "anchor"), (4, 2, "anchor"),
+                                         (2, 1, "anchor"), (2, 2, "anchor"), (4, 1, "dense"),
+                                         (3, 1, "dense"), (4, 2, "sale"), (3, 3, "sale")])
+def test_gqa_group_sizes_single_and_paired_kernels(hq, hkv, mode):
+    """Odd Hq/Hkv runs the one-head-per-CTA kernel, even Hq/Hkv the paired kernel
+    (two q heads share every K/V tile through a tagged union list)."""
+    from workloads import Workload
+    L = 2100
+    w = Workload(f"gqa-{hq}-{hkv}", 9, 1, hq, hkv, L, sink=64, local=256, theta=2.5,
+                 needles_per_head=12)
+    inp = generate(w)
+    heads = [(0, h) for h in range(hq)]
+    if mode == "sale":
+        from gpu_common import compare_sale_masks
+        run = Run(inp, mode="sale", sink=64, local=256, tau=0.02, block_k=32)
+        compare_sale_masks(run, inp, heads)
+    elif mode == "anchor":
+        run = Run(inp, mode="anchor", sink=64, local=256, theta=2.5)
+        compare_anchor_masks(run, inp, heads)
+    else:
+        run = Run(inp, mode="dense", sink=64, local=256)
+    rows = {hd: sample_rows(L, 40, 3 * hd[1] + hq, must=(0, 127, 128, L - 1)) for hd in heads}
+    compare_outputs(run, inp, rows, dense=(mode == "dense"))
+
+
+@pytest.mark.parametrize("step,hq,hkv", [(2, 1, 1), (16, 1, 1), (4, 4, 2), (16, 8, 2)])
+def test_step_grouping(step, hq, hkv):
+    """AnchorAttention's query-block grouping: a key kept by any block of a group
+    of `step` blocks is kept by all of them (within each block's candidates)."""
+    from workloads import Workload
+    L = 6000
+    w = Workload(f"step-{step}-{hq}", 12, 1, hq, hkv, L, sink=64, local=256, theta=2.6,
+                 needles_per_head=16)
+    inp = generate(w)
+    run = Run(inp, mode="anchor", sink=64, local=256, theta=2.6, step=step)
+    heads = [(0, h) for h in range(hq)]
+    compare_anchor_masks(run, inp, heads)
+    rows = {hd: sample_rows(L, 30, 5 * hd[1] + step, must=(L - 1, 2047, 2048)) for hd in heads}
+    compare_outputs(run, inp, rows)

@@ -41,9 +41,9 @@ def test_argument_errors_return_before_launch():
     assert spa.sparse_prefill_plan(p, q, k, 0, workspace_bytes=n) == spa.SPA_ERR_INVALID
     assert spa.sparse_prefill_plan(p, q.data_ptr() + 2, k, ws) == spa.SPA_ERR_INVALID
     assert spa.sparse_prefill_attn(p, q, k, v, ws, 0) == spa.SPA_ERR_INVALID
-    bad = [dict(head_dim=64), dict(causal=0), dict(step=2), dict(local=100), dict(local=64),
+    bad = [dict(head_dim=64), dict(causal=0), dict(step=0), dict(local=100), dict(local=64),
            dict(theta=math.nan)]
-    codes = [spa.SPA_ERR_UNSUPPORTED, spa.SPA_ERR_UNSUPPORTED, spa.SPA_ERR_UNSUPPORTED,
+    codes = [spa.SPA_ERR_UNSUPPORTED, spa.SPA_ERR_UNSUPPORTED, spa.SPA_ERR_INVALID,
              spa.SPA_ERR_INVALID, spa.SPA_ERR_INVALID, spa.SPA_ERR_INVALID]
     for kw, code in zip(bad, codes):
         pb = spa.make_params(1, 1, 1, 1024, **{"sink": 64, "local": 128, **kw})
@@ -55,12 +55,17 @@ def test_argument_errors_return_before_launch():
     assert spa.sparse_prefill_plan(ps, q, k, ws) == spa.SPA_ERR_INVALID
 
 
-def test_bounded_wait_expiry_reports_timeout_and_context_survives():
-    inp, q, k, v = _bufs()
-    p = spa.make_params(1, 1, 1, 1024, sink=64, local=128, theta=3.0,
+@pytest.mark.parametrize("hq", [1, 2])
+def test_bounded_wait_expiry_reports_timeout_and_context_survives(hq):
+    """hq = 1 runs the one-head kernel, hq = 2 the paired kernel."""
+    from workloads import Workload
+    w = Workload(f"stall-{hq}", 11, 1, hq, 1, 1024, sink=64, local=128, needles_per_head=4)
+    inp = generate(w)
+    q, k, v = to_dev(inp.q), to_dev(inp.k), to_dev(inp.v)
+    p = spa.make_params(1, hq, 1, 1024, sink=64, local=128, theta=3.0,
                         wait_limit_us=20000, debug_flags=spa.SPA_DEBUG_STALL_ATTN)
     ws = torch.zeros(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device="cuda")
-    o = torch.zeros((1, 1, 1024, 128), dtype=torch.bfloat16, device="cuda")
+    o = torch.zeros((1, hq, 1024, 128), dtype=torch.bfloat16, device="cuda")
     spa.check(spa.sparse_prefill_plan(p, q, k, ws))
     assert spa.sparse_prefill_attn(p, q, k, v, ws, o) == spa.SPA_OK
     st, s = spa.sparse_prefill_stats(p, ws)
@@ -68,7 +73,7 @@ def test_bounded_wait_expiry_reports_timeout_and_context_survives():
     # the context is still usable: a normal call afterwards succeeds and is correct
     run = Run(inp, mode="anchor", sink=64, local=128, theta=3.0, dev=(q, k, v))
     assert run.stats.error_bits == 0
-    compare_outputs(run, inp, {(0, 0): range(0, 1024, 7)})
+    compare_outputs(run, inp, {(0, h): range(0, 1024, 7) for h in range(hq)})
 
 
 def test_corrupted_list_index_is_caught_in_bounds():

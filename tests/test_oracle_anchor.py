@@ -173,3 +173,33 @@ def test_anchor_head_equals_per_block():
         np.testing.assert_array_equal(many[qb].kept, one.kept)
         np.testing.assert_allclose(many[qb].margin, one.margin, atol=1e-12, rtol=0)
         assert many[qb].xbar_a == one.xbar_a
+
+
+def test_step_grouping_pins():
+    w, qh, kh, _ = _small_case(L=2000)
+    L, bq = 2000, w.block_q
+    nqb = (L + bq - 1) // bq
+    own = osel.anchor_head(qh, kh, range(nqb), bq=bq, sink=w.sink, local=w.local, theta=2.6)
+    sel = lambda b: own[b].kept
+    for qb in range(nqb):
+        geo = osel.block_geometry(qb, L, bq, w.sink, w.local)
+        # step 1 is the identity
+        np.testing.assert_array_equal(
+            osel.step_union(sel, qb, step=1, nqb=nqb, cand_lo=geo.cand_lo, cand_hi=geo.cand_hi),
+            own[qb].kept)
+        # nesting: a block keeps at least its own selection, and more with larger groups
+        # (groups of 2 sit inside groups of 4, which sit inside groups of 16)
+        prev = set(own[qb].kept)
+        for step in (2, 4, 16):
+            cur = set(osel.step_union(sel, qb, step=step, nqb=nqb, cand_lo=geo.cand_lo,
+                                      cand_hi=geo.cand_hi))
+            assert prev <= cur
+            assert all(geo.cand_lo <= j < geo.cand_hi for j in cur)
+            prev = cur
+        # a group covering the whole layer: the union of every block's selection,
+        # clipped to this block's candidates
+        allkeys = np.unique(np.concatenate([own[b].kept for b in range(nqb)]))
+        expect = allkeys[(allkeys >= geo.cand_lo) & (allkeys < geo.cand_hi)]
+        np.testing.assert_array_equal(
+            osel.step_union(sel, qb, step=nqb, nqb=nqb, cand_lo=geo.cand_lo,
+                            cand_hi=geo.cand_hi), expect)
