@@ -35,6 +35,7 @@ class SpaParams(ctypes.Structure):
         ("local", ctypes.c_int32), ("step", ctypes.c_int32), ("mode", ctypes.c_int32),
         ("theta", ctypes.c_float), ("tau", ctypes.c_float), ("softmax_scale", ctypes.c_float),
         ("wait_limit_us", ctypes.c_uint32), ("debug_flags", ctypes.c_uint32),
+        ("tau_per_head", ctypes.POINTER(ctypes.c_float)),
     ]
 
 
@@ -86,13 +87,19 @@ def make_params(batch: int, heads_q: int, heads_kv: int, seq_len: int, *, mode="
                 sink: int = 128, local: int = 256, theta: float = 5.0, tau: float = 1e-3,
                 block_k: Optional[int] = None, softmax_scale: float = 0.0,
                 wait_limit_us: int = 0, debug_flags: int = 0, head_dim: int = 128,
-                causal: int = 1, block_q: int = 128, step: int = 1) -> SpaParams:
+                causal: int = 1, block_q: int = 128, step: int = 1,
+                tau_per_head=None) -> SpaParams:
     m = MODES[mode] if isinstance(mode, str) else int(mode)
     if block_k is None:
         block_k = 32 if m == SPA_MODE_SALE else 1
-    return SpaParams(batch, heads_q, heads_kv, seq_len, head_dim, causal, block_q, block_k,
-                     sink, local, step, m, float(theta), float(tau), float(softmax_scale),
-                     int(wait_limit_us), int(debug_flags))
+    p = SpaParams(batch, heads_q, heads_kv, seq_len, head_dim, causal, block_q, block_k,
+                  sink, local, step, m, float(theta), float(tau), float(softmax_scale),
+                  int(wait_limit_us), int(debug_flags), None)
+    if tau_per_head is not None:
+        arr = (ctypes.c_float * len(tau_per_head))(*[float(t) for t in tau_per_head])
+        p._tau_keepalive = arr          # the struct holds a raw pointer into this array
+        p.tau_per_head = ctypes.cast(arr, ctypes.POINTER(ctypes.c_float))
+    return p
 
 
 def _ptr(x) -> Optional[int]:

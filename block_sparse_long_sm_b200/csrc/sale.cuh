@@ -112,6 +112,7 @@ constexpr uint32_t kIdescI8N64 = make_idesc(2, 1, 128, 64, 0, 0);
 struct SaleArgs {
   int B, Hq, Hkv, L, nqb, group;
   int sink, local, bk, nkb;
+  int bk_log2;              // bk is a power of two
   int chunks;               // ceil(group / kSaleHeads)
   float scale, tau;
   const float* sq;          // [B*Hq][nqb]
@@ -120,6 +121,7 @@ struct SaleArgs {
   int nwords;
   uint32_t* err;
   uint64_t wait_ns;
+  float tau_h[128];         // threshold of each q head (index h), SPA_MAX_TAU_HEADS
 };
 
 __global__ void __launch_bounds__(kSaleThreads, 1)
@@ -263,6 +265,7 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
       if (!warp_wait(bar_afull(bb), (t >> 1) & 1, wc)) break;
       tc_fence_after();
       const int key0 = tile_key0(t);
+      uint32_t gbits = 0;                              // bit 4u + g: head hsel + 2u, group g
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int j = hsel + 2 * u;
@@ -284,7 +287,7 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
               const int col = c * 32 + e;
               const float v = col < limit
                                   ? static_cast<float>(static_cast<int>(sr[c][e])) *
-                                        (cq[u] * kscale[min(key0 + col, a.L - 1) / a.bk])
+                                        (cq[u] * kscale[min(key0 + col, a.L - 1) >> a.bk_log2])
                                   : -INFINITY;
               sr[c][e] = __float_as_uint(v);
               tm = fmaxf(tm, v);
@@ -301,12 +304,12 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
             m[u] = mn;
           }
           if (t == n_stat_t - 1)
-            thr[u] = row_valid ? m[u] + logf(a.tau * l[u]) : INFINITY;   // t_i = em + ln(tau el)
+            thr[u] = row_valid ? m[u] + logf(a.tau_h[h0 + hsel + 2 * u] * l[u])   // t_i = em + ln(tau el)
+                               : INFINITY;
         } else {
           uint32_t pk[32];
           tmem_ld32_pack16(taddr, pk);
           tmem_ld_wait();
-          uint32_t gbits = 0;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {               // 16 keys = 8 packed registers
             const uint32_t* q = pk + 8 * g;
@@ -316,15 +319,23 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
             const int mx = max(static_cast<int>(static_cast<int16_t>(mm & 0xffffu)),
                                static_cast<int>(mm) >> 16);
             const int key = key0 + 16 * g;
-            if (key < cand_hi && static_cast<float>(mx) * (cq[u] * kscale[key / a.bk]) >= thr[u])
-              gbits |= 1u << g;
-          }
-          gbits = __reduce_or_sync(0xffffffffu, gbits);
-          if (lane == 0 && gbits) {
-            const int g0 = (key0 - cand_lo) / 16;    // multiple of 4: one word holds all 4 bits
-            atomicOr(&gflags[j * kMaxGroupWords + (g0 >> 5)], gbits << (g0 & 31));
+            if (key < cand_hi && static_cast<float>(mx) * (cq[u] * kscale[key >> a.bk_log2]) >= thr[u])
+              gbits |= 1u << (4 * u + g);
           }
         }
+      }
+      if (t >= n_stat_t) {
+        // one warp reduction and at most two shared atomics per tile for both heads
+        gbits = __reduce_or_sync(0xffffffffu, gbits);
+        if (lane == 0 && gbits) {
+          const int g0 = (key0 - cand_lo) / 16;      // multiple of 4: one word holds 4 bits
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const uint32_t bits = (gbits >> (4 * u)) & 0xfu;
+            if (bits) atomicOr(&gflags[(hsel + 2 * u) * kMaxGroupWords + (g0 >> 5)], bits << (g0 & 31));
+          }
+        }
+        gbits = 0;
       }
       tc_fence_before();
       mbar_arrive(bar_afree(bb));

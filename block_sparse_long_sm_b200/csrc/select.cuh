@@ -499,18 +499,23 @@ compact_kernel(const CompactArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// two heads' bitmasks -> one ascending union list with membership tags
+// two heads' bitmasks -> both heads' lists + one tagged union list
 // ---------------------------------------------------------------------------
 // For the paired attention kernel (two q heads of one GQA group share every
-// K/V tile): entry = index | (in head 2p) << 30 | (in head 2p+1) << 31.
+// K/V tile).  One pass over the two bitmask rows writes head A's and head
+// B's ascending lists and counts (the documented per-head output, exactly as
+// compact_kernel would) and the union list, whose entries are
+// index | (kept by head 2p) << 30 | (kept by head 2p+1) << 31.
 struct PairCompactArgs {
   int nqb, heads_q, sink, local, unit, step;
   const uint32_t* mask;     // [B*Hq*nqb][nwords]
   int nwords;
-  uint32_t* lists;          // [B*Hq/2][per_head] tagged entries
+  int* lists;               // per-head lists (as compact_kernel)
+  int* counts;              // per-head counts
+  uint32_t* pair_lists;     // [B*Hq/2][per_head] tagged entries
   long long list_per_head;
   long long cap_a;
-  int* counts;              // [B*Hq/2*nqb]
+  int* pair_counts;         // [B*Hq/2*nqb]
 };
 
 __global__ void __launch_bounds__(kCompactThreads)
@@ -518,7 +523,8 @@ pair_compact_kernel(const PairCompactArgs a) {
   const int row = blockIdx.x;                       // (b, pair, qb)
   const int pair = row / a.nqb, qb = row - (row / a.nqb) * a.nqb;
   const int b = pair / (a.heads_q / 2), pp = pair - b * (a.heads_q / 2);
-  const long long rowA = ((long long)b * a.heads_q + 2 * pp) * a.nqb + qb;
+  const int bhA = b * a.heads_q + 2 * pp;
+  const long long rowA = (long long)bhA * a.nqb + qb;
   const long long rowB = rowA + a.nqb;
   const int ls = max(0, (qb + 1) * 128 - a.local);
   const int bit_lo = a.sink / a.unit;
@@ -547,60 +553,86 @@ pair_compact_kernel(const PairCompactArgs a) {
       }
     }
   };
-  uint32_t* out = a.lists + (long long)pair * a.list_per_head + cap_prefix(qb, 128, a.cap_a) / a.unit;
+  const long long off = cap_prefix(qb, 128, a.cap_a) / a.unit;
+  int* outA = a.lists + (long long)bhA * a.list_per_head + off;
+  int* outB = outA + a.list_per_head;
+  uint32_t* outU = a.pair_lists + (long long)pair * a.list_per_head + off;
 
-  __shared__ int warp_cnt[kCompactThreads / 32];
-  __shared__ int warp_base[kCompactThreads / 32];
+  __shared__ int warp_cnt[3][kCompactThreads / 32];
+  __shared__ int warp_base[3][kCompactThreads / 32];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = kCompactThreads / 32;
   const int seg = (((n + nw - 1) / nw) + 31) & ~31;
   const int s_lo = w_lo + warp * seg;
   const int s_hi = min(s_lo + seg, w_hi);
-  int cnt = 0;
+  int ca = 0, cb = 0, cu = 0;
   for (int w = s_lo + lane; w < s_hi; w += 32) {
     uint32_t wa, wb;
     words_at(w, wa, wb);
-    cnt += __popc(wa | wb);
+    ca += __popc(wa);
+    cb += __popc(wb);
+    cu += __popc(wa | wb);
   }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-  if (lane == 0) warp_cnt[warp] = cnt;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int i = 0; i < nw; ++i) {
-      warp_base[i] = run;
-      run += warp_cnt[i];
-    }
-    a.counts[row] = run;
+  for (int o = 16; o > 0; o >>= 1) {
+    ca += __shfl_xor_sync(0xffffffffu, ca, o);
+    cb += __shfl_xor_sync(0xffffffffu, cb, o);
+    cu += __shfl_xor_sync(0xffffffffu, cu, o);
+  }
+  if (lane == 0) {
+    warp_cnt[0][warp] = ca;
+    warp_cnt[1][warp] = cb;
+    warp_cnt[2][warp] = cu;
   }
   __syncthreads();
-  int base = warp_base[warp];
+  if (threadIdx.x < 3) {
+    int run = 0;
+    for (int i = 0; i < nw; ++i) {
+      warp_base[threadIdx.x][i] = run;
+      run += warp_cnt[threadIdx.x][i];
+    }
+    if (threadIdx.x == 0) a.counts[rowA] = run;
+    if (threadIdx.x == 1) a.counts[rowB] = run;
+    if (threadIdx.x == 2) a.pair_counts[row] = run;
+  }
+  __syncthreads();
+  int base_a = warp_base[0][warp], base_b = warp_base[1][warp], base_u = warp_base[2][warp];
   const uint32_t lt = (1u << lane) - 1u;
+  auto scan = [&](int v) {
+    int incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    return incl;
+  };
   for (int w0 = s_lo; w0 < s_hi; w0 += 32) {
     uint32_t wa = 0u, wb = 0u;
     if (w0 + lane < s_hi) words_at(w0 + lane, wa, wb);
-    const uint32_t word = wa | wb;
-    const int pc = __popc(word);
-    int incl = pc;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-    const int excl = incl - pc;
+    const uint32_t wu = wa | wb;
+    const int ia = scan(__popc(wa)), ib = scan(__popc(wb)), iu = scan(__popc(wu));
+    const int ea = ia - __popc(wa), eb = ib - __popc(wb), eu = iu - __popc(wu);
     for (int j = 0; j < 32; ++j) {
-      const uint32_t wj = __shfl_sync(0xffffffffu, word, j);
-      if (wj == 0u) continue;                         // warp-uniform
+      // every shuffle is executed by the whole warp, before any lane-dependent branch
+      const uint32_t uj = __shfl_sync(0xffffffffu, wu, j);
+      if (uj == 0u) continue;                         // warp-uniform
       const uint32_t aj = __shfl_sync(0xffffffffu, wa, j);
       const uint32_t bj = __shfl_sync(0xffffffffu, wb, j);
-      const int oj = __shfl_sync(0xffffffffu, excl, j);
-      if ((wj >> lane) & 1u) {
+      const int ou = __shfl_sync(0xffffffffu, eu, j);
+      const int oa = __shfl_sync(0xffffffffu, ea, j);
+      const int ob = __shfl_sync(0xffffffffu, eb, j);
+      const int key = 32 * (w0 + j) + lane;
+      if ((uj >> lane) & 1u) {
         const uint32_t tag = (((aj >> lane) & 1u) << 30) | (((bj >> lane) & 1u) << 31);
-        out[base + oj + __popc(wj & lt)] = static_cast<uint32_t>(32 * (w0 + j) + lane) | tag;
+        outU[base_u + ou + __popc(uj & lt)] = static_cast<uint32_t>(key) | tag;
       }
+      if ((aj >> lane) & 1u) outA[base_a + oa + __popc(aj & lt)] = key;
+      if ((bj >> lane) & 1u) outB[base_b + ob + __popc(bj & lt)] = key;
     }
-    base += __shfl_sync(0xffffffffu, incl, 31);
+    base_a += __shfl_sync(0xffffffffu, ia, 31);
+    base_b += __shfl_sync(0xffffffffu, ib, 31);
+    base_u += __shfl_sync(0xffffffffu, iu, 31);
   }
 }
 

@@ -65,6 +65,11 @@ spa_status validate(const spa_params* p) {
         return SPA_ERR_UNSUPPORTED;
       if (p->sink % p->block_k != 0) return SPA_ERR_UNSUPPORTED;
       if (!(p->tau > 0.f && p->tau <= 1.f)) return SPA_ERR_INVALID;
+      if (p->tau_per_head) {
+        if (p->heads_q > SPA_MAX_TAU_HEADS) return SPA_ERR_UNSUPPORTED;
+        for (int h = 0; h < p->heads_q; ++h)
+          if (!(p->tau_per_head[h] > 0.f && p->tau_per_head[h] <= 1.f)) return SPA_ERR_INVALID;
+      }
       if (p->seq_len > 262144) return SPA_ERR_UNSUPPORTED;
       break;
     case SPA_MODE_DENSE:
@@ -290,26 +295,31 @@ SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const
       return SPA_ERR_CUDA;
     const int chunks = (lo.group + kSaleHeads - 1) / kSaleHeads;
     SaleArgs sa{B, Hq, Hkv, L, lo.nqb, lo.group, p->sink, p->local, p->block_k, lo.nkb,
-                chunks, scale, p->tau, reinterpret_cast<const float*>(ws + lo.sq),
+                __builtin_ctz((unsigned)p->block_k), chunks, scale, p->tau, reinterpret_cast<const float*>(ws + lo.sq),
                 reinterpret_cast<const float*>(ws + lo.sk),
-                reinterpret_cast<uint32_t*>(ws + lo.mask), lo.nwords, err, wait_ns(p)};
+                reinterpret_cast<uint32_t*>(ws + lo.mask), lo.nwords, err, wait_ns(p), {}};
+    for (int h = 0; h < Hq && h < SPA_MAX_TAU_HEADS; ++h)
+      sa.tau_h[h] = p->tau_per_head ? p->tau_per_head[h] : p->tau;
     if (set_smem(sale_scan_kernel, kSaleSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
     sale_scan_kernel<<<(unsigned)(BKV * lo.nqb * chunks), kSaleThreads, kSaleSmemBytes,
                        stream>>>(tq8, tk8, sa);
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   }
-  CompactArgs ca{(int)lo.nb, lo.nqb, L, p->sink, p->local, lo.unit, p->step,
-                 reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
-                 reinterpret_cast<int*>(ws + lo.lists), lo.list_per_head, lo.cap_a,
-                 reinterpret_cast<int*>(ws + lo.counts)};
-  compact_kernel<<<(unsigned)lo.nb, kCompactThreads, 0, stream>>>(ca);
-  if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   if (lo.paired) {
+    // one pass writes both heads' lists and their tagged union list
     PairCompactArgs pc{lo.nqb, Hq, p->sink, p->local, lo.unit, p->step,
                        reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
+                       reinterpret_cast<int*>(ws + lo.lists), reinterpret_cast<int*>(ws + lo.counts),
                        reinterpret_cast<uint32_t*>(ws + lo.pair_lists), lo.list_per_head, lo.cap_a,
                        reinterpret_cast<int*>(ws + lo.pair_counts)};
     pair_compact_kernel<<<(unsigned)(lo.nb / 2), kCompactThreads, 0, stream>>>(pc);
+    if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
+  } else {
+    CompactArgs ca{(int)lo.nb, lo.nqb, L, p->sink, p->local, lo.unit, p->step,
+                   reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
+                   reinterpret_cast<int*>(ws + lo.lists), lo.list_per_head, lo.cap_a,
+                   reinterpret_cast<int*>(ws + lo.counts)};
+    compact_kernel<<<(unsigned)lo.nb, kCompactThreads, 0, stream>>>(ca);
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   }
   return SPA_OK;

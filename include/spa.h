@@ -107,7 +107,12 @@ typedef struct {
   float softmax_scale;    /* > 0, or 0 for 1/sqrt(head_dim) */
   uint32_t wait_limit_us; /* bound on every device-side wait; 0 -> 250,000 us */
   uint32_t debug_flags;   /* 0 in normal use; SPA_DEBUG_* test hooks */
+  const float* tau_per_head; /* SALE: optional host array of Hq thresholds (one per q head,
+                                each in (0, 1]; Hq <= SPA_MAX_TAU_HEADS), read during
+                                sparse_prefill_plan; NULL -> `tau` for every head */
 } spa_params;
+
+#define SPA_MAX_TAU_HEADS 128
 
 /* Test hook: the attention kernel's MMA warp additionally waits on a barrier
  * that nothing ever signals, so its bounded wait expires after wait_limit_us;

@@ -167,8 +167,17 @@ def compare_sale_masks(run: Run, inputs: Inputs, heads: Sequence[Tuple[int, int]
 
 
 def compare_outputs(run: Run, inputs: Inputs, rows_of: Dict[Tuple[int, int], Iterable[int]],
-                    dense: bool = False) -> Dict[str, float]:
-    """Output parity on the GPU's own kept sets (or dense causal), given rows per head."""
+                    dense: bool = False, bound: str = "stated") -> Dict[str, float]:
+    """Output parity on the GPU's own kept sets (or dense causal), given rows per head.
+
+    ``bound="stated"`` applies the fixed tolerances above.  ``bound="bf16"``
+    applies instead, element by element, the error bound of the kernel's
+    arithmetic, for inputs whose attention is concentrated on a few keys
+    (a strong sink): the probabilities enter the PV product rounded to bf16
+    (relative error <= 2^-8 each) and the output is rounded to bf16, so
+    |dO_i| <= 2^-8 (sum_j p_ij |v_j| / l_i + 2 |O_i|) + 1e-4, where the
+    weighted mean of |v| is the oracle's attention over |V|.
+    """
     p = run.params
     o_gpu = run.o.float().cpu().numpy() if run.o is not None else None
     lse_gpu = run.lse.cpu().numpy() if run.lse is not None else None
@@ -190,12 +199,23 @@ def compare_outputs(run: Run, inputs: Inputs, rows_of: Dict[Tuple[int, int], Ite
                 return cache[qb]
             o_ref, lse_ref = oatt.attend_rows(qh, kh, vh, rows, lambda i: i // 128, sel, bq=128,
                                               sink=p.sink, local=p.local)
-        errs.append(np.abs(o_gpu[b, h, rows].astype(np.float64) - o_ref).ravel())
+        d = np.abs(o_gpu[b, h, rows].astype(np.float64) - o_ref)
+        if bound == "bf16":
+            if dense:
+                w_ref, _ = oatt.dense_causal_rows(qh, kh, np.abs(vh), rows)
+            else:
+                w_ref, _ = oatt.attend_rows(qh, kh, np.abs(vh), rows, lambda i: i // 128, sel,
+                                            bq=128, sink=p.sink, local=p.local)
+            lim = 2.0 ** -8 * (w_ref + 2.0 * np.abs(o_ref)) + 1e-4
+            worst = float(np.max(d / lim))
+            assert worst <= 1.0, (f"b={b} h={h}: error above the bf16 bound", worst)
+        errs.append(d.ravel())
         if lse_gpu is not None:
             lse_err = max(lse_err, float(np.max(np.abs(lse_gpu[b, h, rows] - lse_ref))))
     e = np.concatenate(errs)
     res = dict(max_abs=float(e.max()), mean_abs=float(e.mean()), lse_max=lse_err, n=int(e.size))
-    assert res["max_abs"] <= O_MAX_ABS, res
+    if bound == "stated":
+        assert res["max_abs"] <= O_MAX_ABS, res
     assert res["mean_abs"] <= O_MEAN_ABS, res
     assert res["lse_max"] <= LSE_ABS, res
     return res

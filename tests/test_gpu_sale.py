@@ -58,3 +58,24 @@ def test_sale_c2_full_size_sampled():
     compare_sale_masks(run, inp, heads, blocks_of=lambda b, h: edge_blocks(w.seq_len, 2, h))
     rows = {hd: sample_rows(w.seq_len, 12, hd[1], must=(w.seq_len - 1,)) for hd in heads}
     compare_outputs(run, inp, rows)
+
+
+@pytest.mark.parametrize("hq,tau", [(1, 0.008), (2, 0.008), (2, 0.002), (4, 0.008)])
+def test_sale_strong_sink_local128(hq, tau):
+    """Calibration-style inputs (strong attention sink, planted needles, local
+    window of one block): SALE really prunes here and the heads of a group keep
+    different blocks, so the paired kernel's per-head membership tags matter."""
+    from workloads import calibration_samples
+    L, sink, local = 1024, 64, 128
+    inp = calibration_samples(1, heads_q=hq, heads_kv=1, seq_len=L, sink=sink, local=local)[0]
+    run = Run(inp, mode="sale", sink=sink, local=local, tau=tau, block_k=32)
+    heads = [(0, h) for h in range(hq)]
+    res = compare_sale_masks(run, inp, heads)
+    nqb = L // 128
+    full = sum(max(0, (qb * 128 + 128 - local - sink)) // 32 for qb in range(nqb)) * hq
+    assert res["kept"] < full, "the case must prune"
+    # attention here sits on a few sink keys, so bf16 rounding of the
+    # probabilities is not averaged away: the kernel's own error bound applies
+    compare_outputs(run, inp, {hd: range(L) for hd in heads}, bound="bf16")
+    dense = Run(inp, mode="dense", sink=sink, local=local)
+    compare_outputs(dense, inp, {hd: range(L) for hd in heads}, dense=True, bound="bf16")

@@ -19,6 +19,8 @@ from ``1000 + config id`` and spawned per (b, g)):
 * u ~ uniform random unit vector in R^128 (normalised N(0, I) draw);
 * for each q head of the group: q_i = z + 2u, z ~ N(0, I);
 * k_j = z + 3u for j < 64 (the biased sink region), else k_j = z;
+  (the two bias factors are fields of the workload; the five layer
+  configurations use 2 and 3, calibration samples a stronger sink);
 * v_j = z;
 * needles, drawn after the base tensors, per q head h of the group:
   m ~ U[128, L), j ~ U[64, m) with j distinct within the kv head;
@@ -58,6 +60,8 @@ class Workload:
     needles_per_head: int = 16
     diffuse_kv_heads: Tuple[int, ...] = ()
     head_dim: int = HEAD_DIM
+    q_bias: float = 2.0           # q_i = z + q_bias * u
+    sink_bias: float = 3.0        # k_j = z + sink_bias * u for j < 64
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -153,14 +157,14 @@ def generate(w: Workload, seq_len: Optional[int] = None,
                 if diffuse:
                     qh = rng.standard_normal((L, d), dtype=np.float32) * np.float32(math.sqrt(0.5))
                 else:
-                    qh = rng.standard_normal((L, d), dtype=np.float32) + np.float32(2.0) * u
+                    qh = rng.standard_normal((L, d), dtype=np.float32) + np.float32(w.q_bias) * u
                 qf.append(qh)
             if diffuse:
                 kf = rng.standard_normal((L, d), dtype=np.float32) * np.float32(math.sqrt(0.5))
             else:
                 kf = rng.standard_normal((L, d), dtype=np.float32)
                 nb = min(SINK_BIAS_ROWS, L)
-                kf[:nb] += np.float32(3.0) * u
+                kf[:nb] += np.float32(w.sink_bias) * u
             vf = rng.standard_normal((L, d), dtype=np.float32)
             if not diffuse and L > 128 + 1:
                 used = set()
@@ -189,3 +193,18 @@ def random_bf16(shape, seed: int, scale: float = 1.0, mean: float = 0.0) -> np.n
     rng = np.random.Generator(np.random.PCG64(seed))
     x = rng.standard_normal(shape, dtype=np.float32) * np.float32(scale) + np.float32(mean)
     return f32_to_bf16_bits(x)
+
+
+def calibration_samples(n: int, *, heads_q: int, heads_kv: int, seq_len: int, sink: int,
+                        local: int, first_cid: int = 60, q_bias: float = 8.0,
+                        sink_bias: float = 12.0, diffuse_kv_heads: Tuple[int, ...] = ()):
+    """Stand-ins for SALE's calibration samples (five Retrieve.KV inputs in the
+    paper): independent draws with a strong attention sink and planted needles,
+    so that SALE at tau = 0.008 really prunes and halving tau matters."""
+    out = []
+    for s in range(n):
+        w = Workload(f"calib-{s}", first_cid + s, 1, heads_q, heads_kv, seq_len, sink=sink,
+                     local=local, needles_per_head=8, diffuse_kv_heads=diffuse_kv_heads,
+                     q_bias=q_bias, sink_bias=sink_bias)
+        out.append(generate(w))
+    return out
