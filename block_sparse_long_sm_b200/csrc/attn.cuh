@@ -40,6 +40,7 @@ constexpr uint32_t kTileBytes = 128u * 128u * 2u;       // one 128x128 bf16 tile
 constexpr uint32_t kHalfBytes = kTileBytes / 2u;        // 128 rows x 64 columns
 constexpr uint32_t kAttnSmemBytes =
     1024u + kTileBytes + kAttnStages * 2u * kTileBytes + 256u;
+static_assert(kAttnSmemBytes <= 232448u, "more shared memory than a CTA may use");
 
 // 2^f on [-1/2, 1/2], degree 3, minimax in relative error (max 7.5e-5); the
 // fit is reproduced by csrc/exp2_poly_fit.py.

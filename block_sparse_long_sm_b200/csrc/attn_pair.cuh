@@ -44,6 +44,7 @@ constexpr int kPairThreads = 384;   // 3 warpgroups: softmax A, softmax B, load 
 constexpr uint32_t kPairBarBytes = 1024u;
 constexpr uint32_t kPairSmemBytes =
     1024u + 2u * kTileBytes + (kPairKStages + kPairVStages) * kTileBytes + kPairBarBytes;
+static_assert(kPairSmemBytes <= 232448u, "more shared memory than a CTA may use");
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(

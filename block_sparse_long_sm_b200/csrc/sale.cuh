@@ -107,6 +107,7 @@ constexpr int kMaxGroupWords = 512;          // candidate 16-key groups / 32 (L 
 constexpr int kMaxScales = 16384;            // key blocks per head (L / bk <= 16384)
 constexpr uint32_t kSaleSmemBytes = 1024u + kSaleHeads * kQ8Bytes + kSaleStages * kK8Bytes +
                                     1024u + kSaleHeads * kMaxGroupWords * 4u + kMaxScales * 4u;
+static_assert(kSaleSmemBytes <= 232448u, "more shared memory than a CTA may use");
 constexpr uint32_t kIdescI8N64 = make_idesc(2, 1, 128, 64, 0, 0);
 
 struct SaleArgs {

@@ -12,6 +12,11 @@
 //                        (hi and lo products accumulated in fp32), the
 //                        difference-aware test of Eq. (2) and the candidate
 //                        range check, written as a key bitmask per block.
+//   stripe_select_kernel the scan fused with the compaction (no bitmask):
+//                        per M tile of query blocks, kept keys appended to
+//                        each block's list in key order; used when the
+//                        selection groups fit in a warp (step <= 32, power
+//                        of two).
 //   compact_kernel       per query block: the bitmask's set bits in
 //                        ascending order, written with coalesced warp stores
 //                        into the block's list (Eq. (3): discrete key
@@ -29,6 +34,7 @@ namespace spa {
 constexpr int kPoolThreads = 192;
 constexpr int kPoolStages = 2;
 constexpr uint32_t kPoolSmemBytes = 1024u + kTileBytes + kPoolStages * kTileBytes + 256u;
+static_assert(kPoolSmemBytes <= 232448u, "more shared memory than a CTA may use");
 
 struct PoolArgs {
   int B, Hq, Hkv, L, nqb, group;
@@ -230,6 +236,7 @@ constexpr int kScanStages = 3;
 constexpr int kScanBufs = 4;
 constexpr int kScanTilesPerChunk = 16;
 constexpr uint32_t kScanSmemBytes = 1024u + 2u * kTileBytes + kScanStages * kTileBytes + 512u;
+static_assert(kScanSmemBytes <= 232448u, "more shared memory than a CTA may use");
 
 struct ScanArgs {
   int B, Hq, Hkv, L, nqb, group;
@@ -403,6 +410,306 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------------
+// pooled-score scan fused with compaction: kept-key lists without a bitmask
+// ---------------------------------------------------------------------------
+// One CTA = one M tile of 128 TMEM lanes = 128 query blocks of one q head,
+// or 64 query blocks of each head of a pair (2p, 2p+1) when the attention
+// kernel pairs heads (rows 0-63 head 2p, rows 64-127 head 2p+1: both heads
+// share the kv head, so each K tile feeds both).  The CTA walks every key tile
+// of its candidate range in ascending order and appends each query block's
+// kept keys to the block's list at a running offset, so the lists come out
+// ascending with no intermediate mask.  For a pair it also writes the union
+// of the two heads' kept keys per query block, each entry tagged with the
+// heads that kept it (index | in 2p << 30 | in 2p+1 << 31), and its size:
+// the paired attention kernel's key list.  Selection groups (step > 1) must
+// lie inside one warp: step a power of two <= 32.
+//
+// Warp 0 loads the pooled-Q tile once and the K tiles (4-stage ring); warp 1
+// issues the hi and lo MMAs into four TMEM accumulators; warps 2-17 each own
+// a TMEM lane quadrant and 32 of the 128 columns (one 32-key word per row).
+// Per key tile the sixteen warps exchange their words through shared memory
+// behind a bounded mbarrier wait, so that every thread knows its row's kept
+// count before its word; each warp then stages its rows' (word, list
+// position) pairs and writes the kept keys with one coalesced store per row
+// (a single add per row when all 32 keys are kept).  CTAs are numbered
+// heaviest first (last M tile first), so the block scheduler fills the GPU
+// longest-job-first.
+constexpr int kSelEpiWarps = 16;
+constexpr int kSelThreads = 32 * (2 + kSelEpiWarps);
+constexpr int kSelStages = 4;
+constexpr int kSelBufs = 4;
+constexpr uint32_t kSelBarBytes = 16384u;   // barriers, TMEM slot, word exchange, store staging
+constexpr uint32_t kSelSmemBytes = 1024u + 2u * kTileBytes + kSelStages * kTileBytes + kSelBarBytes;
+static_assert(kSelSmemBytes <= 232448u, "more shared memory than a CTA may use");
+
+struct SelectArgs {
+  int B, Hq, Hkv, L, nqb, group;
+  int sink, local, step;
+  float theta;
+  int heads_per_item;       // 1, or 2 for a head pair
+  int rows_per_head;        // 128 / heads_per_item
+  int n_mt;                 // M tiles per head
+  int n_items_per_mt;       // B * Hq / heads_per_item
+  const float* xbar;        // [B*Hq*nqb]
+  int* lists;
+  long long list_per_head;
+  long long cap_a;
+  int* counts;              // [B*Hq*nqb]
+  int* pair_counts;         // [B*Hq/2*nqb] (pairs only)
+  uint32_t* pair_lists;     // [B*Hq/2][list_per_head] tagged union entries (pairs only)
+  uint32_t* err;
+  uint64_t wait_ns;
+};
+
+__global__ void __launch_bounds__(kSelThreads, 1)
+stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
+                     const __grid_constant__ CUtensorMap tm_k, const SelectArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t s_base = smem_u32(smem);
+  const uint32_t s_a = s_base;                            // hi tile, then lo tile
+  auto s_k = [&](int st) { return s_base + 2u * kTileBytes + st * kTileBytes; };
+  uint8_t* bar_area = smem + 2 * kTileBytes + kSelStages * kTileBytes;
+  const uint32_t b0 = smem_u32(bar_area);
+  const uint32_t bar_a = b0;
+  auto bar_full = [&](int st) { return b0 + 8u * (1 + st); };
+  auto bar_empty = [&](int st) { return b0 + 8u * (1 + kSelStages + st); };
+  auto bar_sfull = [&](int bb) { return b0 + 8u * (1 + 2 * kSelStages + bb); };
+  auto bar_sfree = [&](int bb) { return b0 + 8u * (1 + 2 * kSelStages + kSelBufs + bb); };
+  auto bar_x = [&](int i) { return b0 + 8u * (1 + 2 * kSelStages + 2 * kSelBufs + i); };
+  const uint32_t bar_drain = b0 + 8u * (3 + 2 * kSelStages + 2 * kSelBufs);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 256);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+  uint4* x_words = reinterpret_cast<uint4*>(bar_area + 1024);     // [2][128 rows]: 4 words
+  uint4* stage = reinterpret_cast<uint4*>(bar_area + 5120);       // [16 warps][32 rows], 8 KB
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // item: heaviest M tile first
+  const int mt = a.n_mt - 1 - static_cast<int>(blockIdx.x) / a.n_items_per_mt;
+  const int gi = static_cast<int>(blockIdx.x) % a.n_items_per_mt;
+  const int bh0 = gi * a.heads_per_item;                  // b * Hq + first head
+  const int R = a.rows_per_head;
+  const int qb0 = mt * R;
+  const int qb_last = min(qb0 + R, a.nqb) - 1;
+  const int key_end = max(0, (qb_last + 1) * 128 - a.local);  // ls of the last block
+  const int kt0 = a.sink / 128;
+  const int T = key_end > a.sink ? (key_end + 127) / 128 - kt0 : 0;
+  const int b = bh0 / a.Hq;
+  const int kv_row0 = (b * a.Hkv + (bh0 - b * a.Hq) / a.group) * a.L;
+  const int BH = a.B * a.Hq;
+  const bool paired = a.heads_per_item == 2;
+  // epilogue row of this thread (warps 2-17): TMEM lane r, key word qtr
+  const int quad = warp & 3;
+  const int qtr = (warp - 2) >> 2;               // key columns [32*qtr, 32*qtr + 32)
+  const int r = quad * 32 + lane;
+  const int hs = r / R;                          // head of the pair (0 when unpaired)
+  const int qb = qb0 + (r - hs * R);
+  const int bh = bh0 + hs;
+  const bool row_valid = warp >= 2 && qb < a.nqb;
+  int off = 0;                                   // kept keys written so far (this row)
+  int uoff = 0;                                  // union entries so far (2p+1 rows)
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar_a, 1);
+    for (int st = 0; st < kSelStages; ++st) {
+      mbar_init(bar_full(st), 1);
+      mbar_init(bar_empty(st), 1);
+    }
+    for (int i = 0; i < kSelBufs; ++i) {
+      mbar_init(bar_sfull(i), 1);
+      mbar_init(bar_sfree(i), 32 * kSelEpiWarps);
+    }
+    mbar_init(bar_x(0), 32 * kSelEpiWarps);
+    mbar_init(bar_x(1), 32 * kSelEpiWarps);
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0u;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const WaitCtx wc{abort_flag, a.err, a.wait_ns};
+
+  if (warp == 0) {
+    if (lane == 0 && T > 0) {
+      mbar_arrive_expect_tx(bar_a, 2 * kTileBytes);
+      for (int part = 0; part < 2; ++part)            // hi, then lo
+        for (int h2 = 0; h2 < a.heads_per_item; ++h2) {
+          const uint32_t dst = s_a + part * kTileBytes + h2 * R * 128u;
+          const int plane = part * BH + bh0 + h2;
+          tma_load_3d(dst, &tm_qbar, bar_a, 0, qb0, plane);
+          tma_load_3d(dst + kHalfBytes, &tm_qbar, bar_a, 64, qb0, plane);
+        }
+      int issued = 0;
+      for (int t = 0; t < T; ++t) {
+        const int st = t % kSelStages;
+        if (t >= kSelStages && !mbar_wait(bar_empty(st), ((t / kSelStages) - 1) & 1, wc)) break;
+        const int key0 = (kt0 + t) * 128;
+        mbar_arrive_expect_tx(bar_full(st), kTileBytes);
+        tma_load_2d(s_k(st), &tm_k, bar_full(st), 0, kv_row0 + key0);
+        tma_load_2d(s_k(st) + kHalfBytes, &tm_k, bar_full(st), 64, kv_row0 + key0);
+        issued = t + 1;
+      }
+      {  // no copy may still be in flight when the CTA exits
+        mbar_drain(bar_a, 0, a.wait_ns);
+        for (int t = max(0, issued - kSelStages); t < issued; ++t)
+          mbar_drain(bar_full(t % kSelStages), (t / kSelStages) & 1, a.wait_ns);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && T > 0) {
+      bool ok = mbar_wait(bar_a, 0, wc);
+      for (int t = 0; ok && t < T; ++t) {
+        const int st = t % kSelStages, bb = t % kSelBufs;
+        if (!(ok = mbar_wait(bar_full(st), (t / kSelStages) & 1, wc))) break;
+        if (t >= kSelBufs && !(ok = mbar_wait(bar_sfree(bb), ((t / kSelBufs) - 1) & 1, wc)))
+          break;
+        tc_fence_after();
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {       // hi, then lo
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off8 = (kk >> 2) * kHalfBytes + (kk & 3) * 32u;
+            mma_bf16_ss(tmem + 128u * bb, smem_desc_sw128(s_a + part * kTileBytes + off8, 16),
+                        smem_desc_sw128(s_k(st) + off8, 16), kIdescQK,
+                        (part > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        mma_commit(bar_sfull(bb));
+        mma_commit(bar_empty(st));
+      }
+      mma_commit(bar_drain);
+      mbar_drain(bar_drain, 0, a.wait_ns);
+    }
+    __syncwarp();
+  } else {
+    const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
+    // keep key j  <=>  anchor mean - pooled score <= theta  <=>  score >= xbar - theta
+    const float thr = row_valid ? a.xbar[(long long)bh * a.nqb + qb] - a.theta : INFINITY;
+    const int cand_hi = row_valid ? max(0, (qb + 1) * 128 - a.local) : 0;   // ls of this block
+    // element offset of this row's list inside its head's list region
+    const int row_elem = row_valid ? static_cast<int>(cap_prefix(qb, 128, a.cap_a)) : 0;
+    int* head_lists = a.lists + (long long)bh * a.list_per_head;    // the same for the warp
+    const bool union_row = paired && hs == 1;     // this thread also writes the pair's union
+    uint32_t* pair_list = paired ? a.pair_lists + (long long)(bh0 >> 1) * a.list_per_head : nullptr;
+    const uint32_t lt = (1u << lane) - 1u;
+    uint4* my_stage = stage + (warp - 2) * 32;
+    const uint32_t below_q = (1u << qtr) - 1u;  // words of this row before this warp's
+    for (int t = 0; t < T; ++t) {
+      const int bb = t % kSelBufs, xs = t & 1;
+      if (!warp_wait(bar_sfull(bb), (t / kSelBufs) & 1, wc)) break;
+      tc_fence_after();
+      uint32_t sr[32];
+      tmem_ld32(tmem + lane_off + 128u * bb + 32u * qtr, sr);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(bar_sfree(bb));
+      const int key0 = (kt0 + t) * 128 + 32 * qtr;
+      // candidate keys of this row inside these 32 columns: [lo, hi)
+      const int lo = max(a.sink - key0, 0);
+      const int hi = min(cand_hi - key0, 32);
+      uint32_t part[4] = {0u, 0u, 0u, 0u};             // four independent chains
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        if (__uint_as_float(sr[e]) >= thr) part[e & 3] |= 1u << e;
+      const uint32_t bits = (part[0] | part[1]) | (part[2] | part[3]);
+      uint32_t range = 0;
+      if (hi > lo) range = (hi - lo >= 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u)) << lo;
+      uint32_t w = bits & range;
+      // selection group: OR over the group's rows (neighbouring lanes), each
+      // row cut to its own candidates before and after
+      for (int o = 1; o < a.step; o <<= 1) w |= __shfl_xor_sync(0xffffffffu, w, o);
+      if (a.step > 1) w &= range;
+      reinterpret_cast<uint32_t*>(x_words + xs * 128 + r)[qtr] = w;
+      mbar_arrive(bar_x(xs));
+      if (!warp_wait(bar_x(xs), (t >> 1) & 1, wc)) break;
+      const uint4 mine = x_words[xs * 128 + r];            // this row's four words
+      const uint32_t* mw = &mine.x;
+      int before = 0, total = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c = __popc(mw[q]);
+        before += ((below_q >> q) & 1u) ? c : 0;
+        total += c;
+      }
+      uint32_t awq = 0u;                              // head 2p's word (2p+1 rows)
+      int ubefore = 0, utotal = 0;
+      if (union_row) {
+        const uint4 av = x_words[xs * 128 + (r - 64)];
+        const uint32_t* aw = &av.x;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int cu = __popc(aw[q] | mw[q]);
+          ubefore += ((below_q >> q) & 1u) ? cu : 0;
+          utotal += cu;
+        }
+        awq = qtr == 0 ? av.x : qtr == 1 ? av.y : qtr == 2 ? av.z : av.w;
+      }
+      // append.  When every row of the warp keeps all 32 keys of its word (the
+      // dense case), every row stores the same 32 values: one shuffle and one
+      // coalesced store per row.  Otherwise stage (word, list position[, head
+      // 2p's word, union position]) and store each row's set bits.
+      const int key = key0 + lane;
+      const int pos = row_elem + off + before;
+      const int upos = row_elem + uoff + ubefore;
+      const bool dense = __all_sync(0xffffffffu, w == 0xffffffffu && (!union_row || awq == 0xffffffffu));
+      if (dense) {
+        int* hl = head_lists + lane;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) hl[__shfl_sync(0xffffffffu, pos, j)] = key;
+        if (union_row) {                              // warp-uniform
+          uint32_t* pl = pair_list + lane;
+          const uint32_t both = static_cast<uint32_t>(key) | (3u << 30);
+#pragma unroll 8
+          for (int j = 0; j < 32; ++j) pl[__shfl_sync(0xffffffffu, upos, j)] = both;
+        }
+      } else {
+        my_stage[lane] = make_uint4(w, static_cast<uint32_t>(pos), awq, static_cast<uint32_t>(upos));
+        __syncwarp();
+#pragma unroll 4
+        for (int j = 0; j < 32; ++j) {
+          const uint4 v = my_stage[j];
+          if (v.x == 0xffffffffu) {
+            head_lists[static_cast<int>(v.y) + lane] = key;
+          } else if (v.x != 0u) {
+            if ((v.x >> lane) & 1u) head_lists[static_cast<int>(v.y) + __popc(v.x & lt)] = key;
+          }
+          if (union_row) {                            // warp-uniform
+            const uint32_t u = v.x | v.z;
+            const uint32_t tag = (((v.z >> lane) & 1u) << 30) | (((v.x >> lane) & 1u) << 31);
+            if (u == 0xffffffffu) {
+              pair_list[static_cast<int>(v.w) + lane] = static_cast<uint32_t>(key) | tag;
+            } else if (u != 0u) {
+              if ((u >> lane) & 1u)
+                pair_list[static_cast<int>(v.w) + __popc(u & lt)] = static_cast<uint32_t>(key) | tag;
+            }
+          }
+        }
+        __syncwarp();
+      }
+      uoff += utotal;
+      off += total;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // written even after an abort: a count never exceeds its block's capacity
+  if (warp >= 2 && qtr == 0 && row_valid) {
+    a.counts[(long long)bh * a.nqb + qb] = off;
+    if (paired && hs == 1) a.pair_counts[(long long)(bh0 >> 1) * a.nqb + qb] = uoff;
+  }
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 

@@ -35,9 +35,13 @@ struct Layout {
   size_t counts = 0, lists = 0, xbar = 0, qbar = 0, mask = 0;
   size_t kpart = 0, kmean = 0, q8 = 0, k8 = 0, sq = 0, sk = 0;
   bool paired = false;              // two q heads per attention CTA (Hq / Hkv even)
+  bool fused = false;               // ANCHOR: scan and compaction in one kernel
   size_t pair_counts = 0, pair_lists = 0;
   size_t total = 0;
 };
+
+// The fused ANCHOR selection keeps each selection group inside one warp.
+bool fused_step(int step) { return step >= 1 && step <= 32 && (step & (step - 1)) == 0; }
 
 spa_status validate(const spa_params* p) {
   if (!p) return SPA_ERR_INVALID;
@@ -103,7 +107,8 @@ Layout layout_of(const spa_params* p) {
     lo.lists = take((size_t)bh * lo.list_per_head * 4);
     lo.xbar = take(lo.nb * 4);
     lo.qbar = take((size_t)2 * lo.nb * 128 * 2);
-    lo.mask = take((size_t)lo.nb * lo.nwords * 4);
+    lo.fused = fused_step(p->step);
+    if (!lo.fused) lo.mask = take((size_t)lo.nb * lo.nwords * 4);
   } else if (p->mode == SPA_MODE_SALE) {
     lo.unit = p->block_k;
     lo.nkb = (L + p->block_k - 1) / p->block_k;
@@ -124,7 +129,8 @@ Layout layout_of(const spa_params* p) {
   }
   lo.paired = (lo.group % 2) == 0;
   if (lo.paired && p->mode != SPA_MODE_DENSE) {
-    // union lists of head pairs for the paired attention kernel (opaque scratch)
+    // tagged union lists of head pairs and their sizes, for the paired
+    // attention kernel (opaque scratch)
     lo.pair_counts = take((lo.nb / 2) * 4);
     lo.pair_lists = take((size_t)(bh / 2) * lo.list_per_head * 4);
   }
@@ -260,6 +266,28 @@ SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const
     anchor_pool_kernel<<<(unsigned)lo.nb, kPoolThreads, kPoolSmemBytes, stream>>>(tq, tk, pa);
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
 
+    if (lo.fused) {
+      // scan + compaction in one pass; a head pair shares each CTA's M tile
+      const int hpi = lo.paired ? 2 : 1;
+      const int R = 128 / hpi;
+      const int n_mt = (lo.nqb + R - 1) / R;
+      CUtensorMap tqsel;
+      if (!map_3d(&tqsel, kBF16, 2, ws + lo.qbar, 128, lo.nqb, 2 * BH, 64, (uint32_t)R, kSW128))
+        return SPA_ERR_CUDA;
+      SelectArgs sa{B, Hq, Hkv, L, lo.nqb, lo.group, p->sink, p->local, p->step, p->theta,
+                    hpi, R, n_mt, (int)(BH / hpi),
+                    reinterpret_cast<const float*>(ws + lo.xbar),
+                    reinterpret_cast<int*>(ws + lo.lists), lo.list_per_head, lo.cap_a,
+                    reinterpret_cast<int*>(ws + lo.counts),
+                    lo.paired ? reinterpret_cast<int*>(ws + lo.pair_counts) : nullptr,
+                    lo.paired ? reinterpret_cast<uint32_t*>(ws + lo.pair_lists) : nullptr, err,
+                    wait_ns(p)};
+      if (set_smem(stripe_select_kernel, kSelSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
+      stripe_select_kernel<<<(unsigned)(n_mt * (BH / hpi)), kSelThreads, kSelSmemBytes, stream>>>(
+          tqsel, tk, sa);
+      if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
+      return SPA_OK;
+    }
     const int nmt = (lo.nqb + 127) / 128;
     const int key_end = std::max(0, lo.nqb * 128 - p->local);
     const int kt0 = p->sink / 128;

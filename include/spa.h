@@ -148,7 +148,9 @@ typedef struct {
 SPA_API size_t sparse_prefill_workspace_bytes(const spa_params* p);
 
 /* Selection.  Reads q, k; writes the index lists and counts into workspace.
- * ANCHOR: anchor/pool kernel, pooled-score scan (tensor cores), compaction.
+ * ANCHOR: anchor/pool kernel, then the pooled-score scan (tensor cores) fused
+ *         with the compaction (a separate bitmask pass when step is not a
+ *         power of two <= 32).
  * SALE:   K mean, int4 quantisation of Q and K, sink-local statistics fused
  *         with the int8 tensor-core block scan, compaction.
  * DENSE:  only resets the workspace header. */

@@ -124,7 +124,7 @@ def test_stats_match_oracle_counts():
                                          (3, 1, "dense"), (4, 2, "sale"), (3, 3, "sale")])
 def test_gqa_group_sizes_single_and_paired_kernels(hq, hkv, mode):
     """Odd Hq/Hkv runs the one-head-per-CTA kernel, even Hq/Hkv the paired kernel
-    (two q heads share every K/V tile through a tagged union list)."""
+    (two q heads share every K/V tile; it merges the two heads' lists)."""
     from workloads import Workload
     L = 2100
     w = Workload(f"gqa-{hq}-{hkv}", 9, 1, hq, hkv, L, sink=64, local=256, theta=2.5,
@@ -144,10 +144,13 @@ def test_gqa_group_sizes_single_and_paired_kernels(hq, hkv, mode):
     compare_outputs(run, inp, rows, dense=(mode == "dense"))
 
 
-@pytest.mark.parametrize("step,hq,hkv", [(2, 1, 1), (16, 1, 1), (4, 4, 2), (16, 8, 2)])
+@pytest.mark.parametrize("step,hq,hkv", [(2, 1, 1), (16, 1, 1), (4, 4, 2), (16, 8, 2), (32, 2, 1),
+                                         (3, 4, 2), (5, 1, 1)])
 def test_step_grouping(step, hq, hkv):
     """AnchorAttention's query-block grouping: a key kept by any block of a group
-    of `step` blocks is kept by all of them (within each block's candidates)."""
+    of `step` blocks is kept by all of them (within each block's candidates).
+    Powers of two up to 32 run the fused scan + compaction kernel, other steps
+    the bitmask + compaction pair."""
     from workloads import Workload
     L = 6000
     w = Workload(f"step-{step}-{hq}", 12, 1, hq, hkv, L, sink=64, local=256, theta=2.6,
