@@ -30,14 +30,13 @@
 // TMEM columns: S0 [0,128)  S1 [128,256)  O [256,384)  P0 [384,448)  P1 [448,512).
 #pragma once
 
+#include "common.cuh"
 #include "ptx.cuh"
 
 namespace spa {
 
 constexpr int kAttnStages = 3;
 constexpr int kAttnThreads = 192;
-constexpr uint32_t kTileBytes = 128u * 128u * 2u;       // one 128x128 bf16 tile
-constexpr uint32_t kHalfBytes = kTileBytes / 2u;        // 128 rows x 64 columns
 constexpr uint32_t kAttnSmemBytes =
     1024u + kTileBytes + kAttnStages * 2u * kTileBytes + 256u;
 static_assert(kAttnSmemBytes <= 232448u, "more shared memory than a CTA may use");
@@ -64,8 +63,6 @@ __device__ __forceinline__ float poly_exp2(float x) {
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
-enum : int { kModeAnchor = 0, kModeSale = 1, kModeDense = 2 };
-
 struct AttnArgs {
   int B, Hq, Hkv, L, nqb, group;
   int sink, local;
@@ -78,6 +75,7 @@ struct AttnArgs {
   int list_unit;              // 1 (keys) or bk (SALE: list holds key-block ids)
   const int* pair_counts;     // paired kernel: union entries per (b, head pair, qb)
   const uint32_t* pair_lists; // paired kernel: tagged union lists
+  const int* pair_split;      // paired kernel: union entries shared with head A's list
   long long pair_per_head;    // list elements per (b, head pair)
   __nv_bfloat16* o;
   float* lse;
@@ -85,15 +83,6 @@ struct AttnArgs {
   uint64_t wait_ns;
   uint32_t debug;
 };
-
-// sum_{q < n} max(0, (q+1)*bq - A): closed-form prefix of the per-block
-// candidate capacity max(0, ls_q - sink) with A = local + sink.
-__host__ __device__ __forceinline__ long long cap_prefix(long long n, long long bq, long long A) {
-  long long q0 = A / bq;
-  if (n <= q0) return 0;
-  long long cnt = n - q0;
-  return bq * ((n * (n + 1) - q0 * (q0 + 1)) / 2) - cnt * A;
-}
 
 struct AttnItem {
   int b, h, kvh, qb, row0, le, ls, sink_end;

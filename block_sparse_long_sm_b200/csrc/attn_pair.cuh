@@ -6,9 +6,10 @@
 // the exponentials of one head overlap the tensor-core work of the other:
 //
 //   * one CTA = (b, kv head, query block, head pair (2p, 2p+1)); the key
-//     sequence is sink tiles, the tiles of the pair's *union* list (plan's
-//     pair_compact_kernel: every entry carries which of the two heads kept
-//     it), and local tiles;
+//     sequence is sink tiles, the tiles of the pair's *union* list (every
+//     entry carries which of the two heads kept it; up to the first entry
+//     where the heads differ the union is head A's own list), and local
+//     tiles;
 //   * warp 8 loads Q of both heads once and K/V tiles into rings of 3 (K) and
 //     2 (V) stages, gathering selected rows with TMA gather4, and publishes a
 //     128-bit membership mask per head for each selected tile;
@@ -74,6 +75,8 @@ __device__ __forceinline__ void tmem_st32_halves(uint32_t taddr, const uint32_t*
 struct PairItem {
   AttnItem it;     // geometry; it.h is head A, it.n_sel counts union keys
   int pair;        // b * Hq / 2 + hA / 2
+  int split;       // union entries before the two heads' lists first differ
+  long long a_off; // head A's list of this block: the union's first `split` entries
 };
 
 __device__ __forceinline__ PairItem pair_item(const AttnArgs& a, int x) {
@@ -93,6 +96,8 @@ __device__ __forceinline__ PairItem pair_item(const AttnArgs& a, int x) {
   it.le = min(it.row0 + 128, a.L);
   it.ls = max(0, it.row0 + 128 - a.local);
   it.sink_end = min(a.sink, it.ls);
+  pi.split = 0;
+  pi.a_off = 0;
   if (a.mode == kModeDense) {
     it.n_sink_t = 0;
     it.n_sel = 0;
@@ -105,6 +110,9 @@ __device__ __forceinline__ PairItem pair_item(const AttnArgs& a, int x) {
     it.loc_start = it.ls;
     it.list_off = (long long)pi.pair * a.pair_per_head +
                   cap_prefix(it.qb, 128, a.cap_a) / a.list_unit;
+    pi.split = a.pair_split[(long long)pi.pair * a.nqb + it.qb];
+    pi.a_off = ((long long)it.b * a.Hq + it.h) * a.list_per_head +
+               cap_prefix(it.qb, 128, a.cap_a) / a.list_unit;
   }
   it.n_sel_t = (it.n_sel + 127) / 128;
   it.n_loc_t = (it.le - it.loc_start + 127) / 128;
@@ -112,9 +120,16 @@ __device__ __forceinline__ PairItem pair_item(const AttnArgs& a, int x) {
 }
 
 // Union entry of selected ordinal n: key index and 2-bit membership tag.
-__device__ __forceinline__ void pair_sel(const AttnArgs& a, const AttnItem& it, int n, int& key,
+// While the two heads' lists agree, the union is head A's list (both heads
+// keep every entry); the plan writes union entries only from the first
+// difference on.
+__device__ __forceinline__ void pair_sel(const AttnArgs& a, const PairItem& pi, int n, int& key,
                                          uint32_t& tag) {
-  const uint32_t e = a.pair_lists[it.list_off + n / a.list_unit];
+  const int ne = n / a.list_unit;
+  const bool shared = ne < pi.split;
+  const uint32_t* src = shared ? reinterpret_cast<const uint32_t*>(a.lists) + pi.a_off
+                               : a.pair_lists + pi.it.list_off;
+  const uint32_t e = src[ne] | (shared ? (3u << 30) : 0u);
   tag = e >> 30;
   const int idx = static_cast<int>(e & 0x3FFFFFFFu);
   key = a.list_unit == 1 ? idx : idx * a.list_unit + n % a.list_unit;
@@ -223,12 +238,12 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (!td.gather) return;
       int first;
       uint32_t ftag;
-      pair_sel(a, it, td.key0, first, ftag);
+      pair_sel(a, pi, td.key0, first, ftag);
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int row = lane * 4 + r;
         if (row < td.valid) {
-          pair_sel(a, it, td.key0 + row, j[r], tg[r]);
+          pair_sel(a, pi, td.key0 + row, j[r], tg[r]);
         } else {
           j[r] = first;
           tg[r] = 0u;

@@ -18,12 +18,10 @@
 //       the integer part.  Output: one bit per key block.
 #pragma once
 
-#include "attn.cuh"
+#include "common.cuh"
 #include "ptx.cuh"
 
 namespace spa {
-
-constexpr int kKmeanChunks = 64;
 
 struct KmeanArgs {
   const __nv_bfloat16* k;   // [B*Hkv][L][128]

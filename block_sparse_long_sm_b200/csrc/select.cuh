@@ -23,7 +23,7 @@
 //                        coordinates), plus the count.
 #pragma once
 
-#include "attn.cuh"
+#include "common.cuh"
 #include "ptx.cuh"
 
 namespace spa {
@@ -31,9 +31,23 @@ namespace spa {
 // ---------------------------------------------------------------------------
 // anchor + pooling
 // ---------------------------------------------------------------------------
-constexpr int kPoolThreads = 192;
-constexpr int kPoolStages = 2;
-constexpr uint32_t kPoolSmemBytes = 1024u + kTileBytes + kPoolStages * kTileBytes + 256u;
+// One CTA streams kPoolQbs consecutive query blocks of one q head: warp 0
+// loads each block's Q tile (2-stage ring) and its sink and local K tiles
+// (3-stage ring); warp 1 issues S = Q K^T per key tile into four TMEM
+// accumulators; warps 2-9 (two per TMEM lane quadrant, 64 columns each)
+// take the causal row max of every tile and, from the Q tile in shared
+// memory, the column sums of the block's rows (each warp pair half the
+// rows).  Per block the two halves are combined through shared memory
+// behind a bounded mbarrier wait: x_a = max * scale, its mean over the
+// block's rows, and avgpool(Q) * scale split into bf16 hi + lo.
+constexpr int kPoolQbs = 8;
+constexpr int kPoolThreads = 320;
+constexpr int kPoolQStages = 2;
+constexpr int kPoolKStages = 3;
+constexpr int kPoolBufs = 4;
+constexpr uint32_t kPoolBarBytes = 8192u;
+constexpr uint32_t kPoolSmemBytes =
+    1024u + (kPoolQStages + kPoolKStages) * kTileBytes + kPoolBarBytes;
 static_assert(kPoolSmemBytes <= 232448u, "more shared memory than a CTA may use");
 
 struct PoolArgs {
@@ -44,6 +58,7 @@ struct PoolArgs {
   __nv_bfloat16* qbar;          // [2][B*Hq][nqb][128]: hi then lo
   uint32_t* err;
   uint64_t wait_ns;
+  int groups;                   // ceil(nqb / kPoolQbs)
 };
 
 __global__ void __launch_bounds__(kPoolThreads, 1)
@@ -53,37 +68,65 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t s_base = smem_u32(smem);
-  const uint32_t s_q = s_base;
-  auto s_k = [&](int st) { return s_base + kTileBytes + st * kTileBytes; };
-  uint8_t* bar_area = smem + kTileBytes + kPoolStages * kTileBytes;
+  auto s_q = [&](int st) { return s_base + st * kTileBytes; };
+  auto s_k = [&](int st) { return s_base + (kPoolQStages + st) * kTileBytes; };
+  uint8_t* bar_area = smem + (kPoolQStages + kPoolKStages) * kTileBytes;
   const uint32_t b0 = smem_u32(bar_area);
-  const uint32_t bar_q = b0;
-  auto bar_full = [&](int s) { return b0 + 8u * (1 + s); };
-  auto bar_empty = [&](int s) { return b0 + 8u * (1 + kPoolStages + s); };
-  const uint32_t bar_sfull0 = b0 + 8u * (1 + 2 * kPoolStages);
-  const uint32_t bar_sfree0 = bar_sfull0 + 16u;
-  const uint32_t bar_drain = bar_sfull0 + 32u;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 8 * (1 + 2 * kPoolStages) + 40);
+  auto bar_qfull = [&](int s) { return b0 + 8u * s; };
+  auto bar_qempty = [&](int s) { return b0 + 8u * (2 + s); };
+  auto bar_kfull = [&](int s) { return b0 + 8u * (4 + s); };
+  auto bar_kempty = [&](int s) { return b0 + 8u * (7 + s); };
+  auto bar_sfull = [&](int s) { return b0 + 8u * (10 + s); };
+  auto bar_sfree = [&](int s) { return b0 + 8u * (14 + s); };
+  auto bar_x = [&](int s) { return b0 + 8u * (18 + s); };       // halves combined
+  auto bar_r = [&](int s) { return b0 + 8u * (20 + s); };       // row sums per quadrant
+  const uint32_t bar_drain = b0 + 8u * 22;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 256);
   volatile uint32_t* abort_flag = tmem_holder + 1;
-  float* red = reinterpret_cast<float*>(tmem_holder + 2);   // 4 partial sums
+  float* x_max = reinterpret_cast<float*>(bar_area + 512);      // [2][2 halves][128]
+  float* x_col = reinterpret_cast<float*>(bar_area + 2560);     // [2][2 halves][128]
+  float* x_red = reinterpret_cast<float*>(bar_area + 4608);     // [2][4 quadrants]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = static_cast<int>(blockIdx.x) / a.groups;
+  const int grp = static_cast<int>(blockIdx.x) - bh * a.groups;
+  const int qb0 = grp * kPoolQbs;
+  const int nq = min(kPoolQbs, a.nqb - qb0);
+  const int b = bh / a.Hq, h = bh - b * a.Hq;
+  const int kv_row0 = (b * a.Hkv + h / a.group) * a.L;
+  // tiles of block qb: sink tiles [0, sink_end), then local tiles [ls, le)
+  auto geom = [&](int qb, int& ls, int& le, int& sink_end, int& n_sink_t, int& T) {
+    const int row0 = qb * 128;
+    le = min(row0 + 128, a.L);
+    ls = max(0, row0 + 128 - a.local);
+    sink_end = min(a.sink, ls);
+    n_sink_t = (sink_end + 127) / 128;
+    T = n_sink_t + (le - ls + 127) / 128;
+  };
+
   if (threadIdx.x == 0) {
-    mbar_init(bar_q, 1);
-    for (int s = 0; s < kPoolStages; ++s) {
-      mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
+    for (int s = 0; s < kPoolQStages; ++s) {
+      mbar_init(bar_qfull(s), 1);
+      mbar_init(bar_qempty(s), 1 + 256);            // the MMAs' commit + every epilogue thread
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar_sfull0 + 8u * i, 1);
-      mbar_init(bar_sfree0 + 8u * i, 128);
+    for (int s = 0; s < kPoolKStages; ++s) {
+      mbar_init(bar_kfull(s), 1);
+      mbar_init(bar_kempty(s), 1);
+    }
+    for (int s = 0; s < kPoolBufs; ++s) {
+      mbar_init(bar_sfull(s), 1);
+      mbar_init(bar_sfree(s), 256);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_x(s), 256);
+      mbar_init(bar_r(s), 128);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), 256);
+    tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -92,60 +135,65 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t tmem = *tmem_holder;
   const WaitCtx wc{abort_flag, a.err, a.wait_ns};
 
-  // block geometry
-  const int x = blockIdx.x;
-  const int bh = x / a.nqb, qb = x - (x / a.nqb) * a.nqb;
-  const int b = bh / a.Hq, h = bh - b * a.Hq;
-  const int kvh = h / a.group;
-  const int row0 = qb * 128;
-  const int le = min(row0 + 128, a.L);
-  const int nrows = le - row0;
-  const int ls = max(0, row0 + 128 - a.local);
-  const int sink_end = min(a.sink, ls);
-  const int n_sink_t = (sink_end + 127) / 128;
-  const int n_loc_t = (le - ls + 127) / 128;
-  const int T = n_sink_t + n_loc_t;
-  const int kv_row0 = (b * a.Hkv + kvh) * a.L;
-  auto tile_key0 = [&](int t) { return t < n_sink_t ? t * 128 : ls + (t - n_sink_t) * 128; };
-
   if (warp == 0) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(bar_q, kTileBytes);
-      const int qrow = bh * a.L + row0;
-      tma_load_2d(s_q, &tm_q, bar_q, 0, qrow);
-      tma_load_2d(s_q + kHalfBytes, &tm_q, bar_q, 64, qrow);
-      int issued = 0;
-      for (int t = 0; t < T; ++t) {
-        const int st = t % kPoolStages;
-        if (t >= kPoolStages && !mbar_wait(bar_empty(st), ((t / kPoolStages) - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(bar_full(st), kTileBytes);
-        tma_load_2d(s_k(st), &tm_k, bar_full(st), 0, kv_row0 + tile_key0(t));
-        tma_load_2d(s_k(st) + kHalfBytes, &tm_k, bar_full(st), 64, kv_row0 + tile_key0(t));
-        issued = t + 1;
+      int gk = 0, issued_q = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < nq; ++i) {
+        const int qb = qb0 + i, qs = i % kPoolQStages;
+        int ls, le, sink_end, n_sink_t, T;
+        geom(qb, ls, le, sink_end, n_sink_t, T);
+        if (i >= kPoolQStages &&
+            !(ok = mbar_wait(bar_qempty(qs), ((i / kPoolQStages) - 1) & 1, wc)))
+          break;
+        mbar_arrive_expect_tx(bar_qfull(qs), kTileBytes);
+        const int qrow = bh * a.L + qb * 128;
+        tma_load_2d(s_q(qs), &tm_q, bar_qfull(qs), 0, qrow);
+        tma_load_2d(s_q(qs) + kHalfBytes, &tm_q, bar_qfull(qs), 64, qrow);
+        issued_q = i + 1;
+        for (int t = 0; t < T; ++t, ++gk) {
+          const int ks = gk % kPoolKStages;
+          if (gk >= kPoolKStages &&
+              !(ok = mbar_wait(bar_kempty(ks), ((gk / kPoolKStages) - 1) & 1, wc)))
+            break;
+          const int key0 = t < n_sink_t ? t * 128 : ls + (t - n_sink_t) * 128;
+          mbar_arrive_expect_tx(bar_kfull(ks), kTileBytes);
+          tma_load_2d(s_k(ks), &tm_k, bar_kfull(ks), 0, kv_row0 + key0);
+          tma_load_2d(s_k(ks) + kHalfBytes, &tm_k, bar_kfull(ks), 64, kv_row0 + key0);
+        }
       }
-      {  // no copy may still be in flight when the CTA exits
-        mbar_drain(bar_q, 0, a.wait_ns);
-        for (int t = max(0, issued - kPoolStages); t < issued; ++t)
-          mbar_drain(bar_full(t % kPoolStages), (t / kPoolStages) & 1, a.wait_ns);
-      }
+      // no copy may still be in flight when the CTA exits
+      for (int i = max(0, issued_q - kPoolQStages); i < issued_q; ++i)
+        mbar_drain(bar_qfull(i % kPoolQStages), (i / kPoolQStages) & 1, a.wait_ns);
+      for (int g = max(0, gk - kPoolKStages); g < gk; ++g)
+        mbar_drain(bar_kfull(g % kPoolKStages), (g / kPoolKStages) & 1, a.wait_ns);
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
-      bool ok = mbar_wait(bar_q, 0, wc);
-      for (int t = 0; ok && t < T; ++t) {
-        const int st = t % kPoolStages, bb = t & 1;
-        if (!(ok = mbar_wait(bar_full(st), (t / kPoolStages) & 1, wc))) break;
-        if (t >= 2 && !(ok = mbar_wait(bar_sfree0 + 8u * bb, ((t - 2) >> 1) & 1, wc))) break;
-        tc_fence_after();
+      int gk = 0;
+      bool ok = true;
+      for (int i = 0; ok && i < nq; ++i) {
+        const int qb = qb0 + i, qs = i % kPoolQStages;
+        int ls, le, sink_end, n_sink_t, T;
+        geom(qb, ls, le, sink_end, n_sink_t, T);
+        if (!(ok = mbar_wait(bar_qfull(qs), (i / kPoolQStages) & 1, wc))) break;
+        for (int t = 0; t < T; ++t, ++gk) {
+          const int ks = gk % kPoolKStages, bb = gk % kPoolBufs;
+          if (!(ok = mbar_wait(bar_kfull(ks), (gk / kPoolKStages) & 1, wc))) break;
+          if (gk >= kPoolBufs && !(ok = mbar_wait(bar_sfree(bb), ((gk / kPoolBufs) - 1) & 1, wc)))
+            break;
+          tc_fence_after();
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks >> 2) * kHalfBytes + (ks & 3) * 32u;
-          mma_bf16_ss(tmem + 128u * bb, smem_desc_sw128(s_q + off, 16),
-                      smem_desc_sw128(s_k(st) + off, 16), kIdescQK, ks > 0 ? 1u : 0u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32u;
+            mma_bf16_ss(tmem + 128u * bb, smem_desc_sw128(s_q(qs) + off, 16),
+                        smem_desc_sw128(s_k(ks) + off, 16), kIdescQK, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_sfull(bb));
+          mma_commit(bar_kempty(ks));
         }
-        mma_commit(bar_sfull0 + 8u * bb);
-        mma_commit(bar_empty(st));
+        if (ok) mma_commit(bar_qempty(qs));            // Q no longer read by the MMAs
       }
       mma_commit(bar_drain);
       mbar_drain(bar_drain, 0, a.wait_ns);
@@ -153,76 +201,98 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
     __syncwarp();
   } else {
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;
+    const int half = (warp - 2) >> 2;              // columns [64 half, 64 half + 64), rows likewise
+    const int r = quad * 32 + lane;                // TMEM lane = query row; also the Q column summed
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    float mx = -INFINITY;
-    bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int bb = t & 1;
-      if (!(ok = warp_wait(bar_sfull0 + 8u * bb, (t >> 1) & 1, wc))) break;
-      tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + 128u * bb + 32u * c, sr[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar_sfree0 + 8u * bb);
-      const int key0 = tile_key0(t);
-      // valid keys: sink tiles below sink_end; local tiles causal (j <= i) and below L
-      int limit = (t < n_sink_t) ? (sink_end - key0) : min(le - key0, row0 + r - key0 + 1);
-      limit = min(limit, 128);
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (c * 32 + e < limit) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
-    }
-    if (ok) {
-      const bool valid = r < nrows;
-      float xa = valid ? mx * a.scale : 0.f;
-      float s = xa;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (lane == 0) red[quad] = s;
-    }
-    // pooled query: thread r owns column d = r (Q is read from shared memory,
-    // so wait on its barrier as well)
-    if (ok) ok = warp_wait(bar_q, 0, wc);
-    if (ok) {
-      float acc = 0.f;
-      const int d = r;
-      const uint32_t half = (d >> 6) * kHalfBytes;
-      const uint32_t byte = (d & 63) * 2;
+    const uint32_t dhalf = (r >> 6) * kHalfBytes;  // Q column r: 64-column half and byte offset
+    const uint32_t dbyte = (r & 63) * 2;
+    int gb = 0;
+    for (int i = 0; i < nq; ++i) {
+      const int qb = qb0 + i, qs = i % kPoolQStages, xs = i & 1;
+      int ls, le, sink_end, n_sink_t, T;
+      geom(qb, ls, le, sink_end, n_sink_t, T);
+      const int row0 = qb * 128;
+      const int nrows = le - row0;
+      // column sum of Q over this half's rows
+      if (!warp_wait(bar_qfull(qs), (i / kPoolQStages) & 1, wc)) break;
+      const uint8_t* qt = smem + (s_q(qs) - s_base);
       auto qv = [&](int rr) {
         return __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16*>(smem + half + sw128_offset(rr, byte)));
+            *reinterpret_cast<const __nv_bfloat16*>(qt + dhalf + sw128_offset(rr, dbyte)));
       };
       float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;   // four independent chains
-      int rr = 0;
-      for (; rr + 4 <= nrows; rr += 4) {
+      const int r_lo = 64 * half, r_hi = min(r_lo + 64, nrows);
+      int rr = r_lo;
+      for (; rr + 4 <= r_hi; rr += 4) {
         p0 += qv(rr);
         p1 += qv(rr + 1);
         p2 += qv(rr + 2);
         p3 += qv(rr + 3);
       }
-      for (; rr < nrows; ++rr) p0 += qv(rr);
-      acc = (p0 + p1) + (p2 + p3);
-      const float qbar = (acc / static_cast<float>(nrows)) * a.scale;
-      const __nv_bfloat16 hi = __float2bfloat16_rn(qbar);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(qbar - __bfloat162float(hi));
-      const long long base = ((long long)bh * a.nqb + qb) * 128 + d;
-      const long long lo_off = (long long)a.B * a.Hq * a.nqb * 128;
-      a.qbar[base] = hi;
-      a.qbar[lo_off + base] = lo;
+      for (; rr < r_hi; ++rr) p0 += qv(rr);
+      const float col = (p0 + p1) + (p2 + p3);
+      mbar_arrive(bar_qempty(qs));
+      // causal row max over this half's columns of the block's key tiles
+      float mx = -INFINITY;
+      bool ok = true;
+      for (int t = 0; t < T; ++t, ++gb) {
+        const int bb = gb % kPoolBufs;
+        if (!(ok = warp_wait(bar_sfull(bb), (gb / kPoolBufs) & 1, wc))) break;
+        tc_fence_after();
+        uint32_t sr[2][32];
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+          tmem_ld32(tmem + lane_off + 128u * bb + 64u * half + 32u * c, sr[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(bar_sfree(bb));
+        const int key0 = (t < n_sink_t ? t * 128 : ls + (t - n_sink_t) * 128) + 64 * half;
+        // valid keys: sink tiles below sink_end; local tiles causal (j <= i) and below L
+        int limit = (t < n_sink_t) ? (sink_end - key0) : min(le - key0, row0 + r - key0 + 1);
+        limit = max(0, min(limit, 64));
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e < limit) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sr[c][e]));
+        mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+      }
+      if (!ok) break;
+      // combine the two halves
+      x_max[(xs * 2 + half) * 128 + r] = mx;
+      x_col[(xs * 2 + half) * 128 + r] = col;
+      mbar_arrive(bar_x(xs));
+      if (!warp_wait(bar_x(xs), (i >> 1) & 1, wc)) break;
+      if (half == 0) {
+        const float m = fmaxf(x_max[(xs * 2) * 128 + r], x_max[(xs * 2 + 1) * 128 + r]);
+        float s = r < nrows ? m * a.scale : 0.f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) x_red[xs * 4 + quad] = s;
+        mbar_arrive(bar_r(xs));
+        if (!warp_wait(bar_r(xs), (i >> 1) & 1, wc)) break;
+        if (r == 0)
+          a.xbar[(long long)bh * a.nqb + qb] =
+              (x_red[xs * 4 + 0] + x_red[xs * 4 + 1] + x_red[xs * 4 + 2] + x_red[xs * 4 + 3]) /
+              static_cast<float>(nrows);
+      } else {
+        // pooled query, column d = r
+        const float sum = x_col[(xs * 2) * 128 + r] + x_col[(xs * 2 + 1) * 128 + r];
+        const float qbar = (sum / static_cast<float>(nrows)) * a.scale;
+        const __nv_bfloat16 hi = __float2bfloat16_rn(qbar);
+        const __nv_bfloat16 lo = __float2bfloat16_rn(qbar - __bfloat162float(hi));
+        const long long base = ((long long)bh * a.nqb + qb) * 128 + r;
+        const long long lo_off = (long long)a.B * a.Hq * a.nqb * 128;
+        a.qbar[base] = hi;
+        a.qbar[lo_off + base] = lo;
+      }
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (threadIdx.x == 64 && !*abort_flag) {
-    a.xbar[(long long)bh * a.nqb + qb] = (red[0] + red[1] + red[2] + red[3]) / static_cast<float>(nrows);
-  }
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 256);
+  if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------------
@@ -461,6 +531,7 @@ struct SelectArgs {
   int* counts;              // [B*Hq*nqb]
   int* pair_counts;         // [B*Hq/2*nqb] (pairs only)
   uint32_t* pair_lists;     // [B*Hq/2][list_per_head] tagged union entries (pairs only)
+  int* pair_split;          // [B*Hq/2*nqb]: union entries before the heads first differ
   uint32_t* err;
   uint64_t wait_ns;
 };
@@ -513,6 +584,7 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
   const bool row_valid = warp >= 2 && qb < a.nqb;
   int off = 0;                                   // kept keys written so far (this row)
   int uoff = 0;                                  // union entries so far (2p+1 rows)
+  int split = -1;                                // union entries before the heads differ
 
   if (threadIdx.x == 0) {
     mbar_init(bar_a, 1);
@@ -645,47 +717,57 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
       }
       uint32_t awq = 0u;                              // head 2p's word (2p+1 rows)
       int ubefore = 0, utotal = 0;
+      bool write_union = false;
       if (union_row) {
         const uint4 av = x_words[xs * 128 + (r - 64)];
         const uint32_t* aw = &av.x;
+        // While the two heads agree, the union is head 2p's list; union
+        // entries are written from the first differing word on.
+        const bool diverged = split >= 0;
+        int first_diff = 4, ucount = 0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int cu = __popc(aw[q] | mw[q]);
+          if (first_diff == 4 && aw[q] != mw[q]) {
+            first_diff = q;
+            if (!diverged) split = uoff + ucount;
+          }
+          ucount += cu;
           ubefore += ((below_q >> q) & 1u) ? cu : 0;
           utotal += cu;
         }
+        write_union = diverged || first_diff <= qtr;
         awq = qtr == 0 ? av.x : qtr == 1 ? av.y : qtr == 2 ? av.z : av.w;
       }
       // append.  When every row of the warp keeps all 32 keys of its word (the
       // dense case), every row stores the same 32 values: one shuffle and one
-      // coalesced store per row.  Otherwise stage (word, list position[, head
-      // 2p's word, union position]) and store each row's set bits.
+      // coalesced store per row.  Otherwise, and for union entries, stage
+      // (word, list position, head 2p's word, union position or none) and
+      // store each row's set bits.
       const int key = key0 + lane;
       const int pos = row_elem + off + before;
-      const int upos = row_elem + uoff + ubefore;
-      const bool dense = __all_sync(0xffffffffu, w == 0xffffffffu && (!union_row || awq == 0xffffffffu));
+      const bool dense = __all_sync(0xffffffffu, w == 0xffffffffu);
       if (dense) {
         int* hl = head_lists + lane;
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) hl[__shfl_sync(0xffffffffu, pos, j)] = key;
-        if (union_row) {                              // warp-uniform
-          uint32_t* pl = pair_list + lane;
-          const uint32_t both = static_cast<uint32_t>(key) | (3u << 30);
-#pragma unroll 8
-          for (int j = 0; j < 32; ++j) pl[__shfl_sync(0xffffffffu, upos, j)] = both;
-        }
-      } else {
-        my_stage[lane] = make_uint4(w, static_cast<uint32_t>(pos), awq, static_cast<uint32_t>(upos));
+      }
+      if (!dense || __any_sync(0xffffffffu, write_union)) {
+        my_stage[lane] = make_uint4(w, static_cast<uint32_t>(pos), awq,
+                                    write_union ? static_cast<uint32_t>(row_elem + uoff + ubefore)
+                                                : 0xffffffffu);
         __syncwarp();
 #pragma unroll 4
         for (int j = 0; j < 32; ++j) {
           const uint4 v = my_stage[j];
-          if (v.x == 0xffffffffu) {
-            head_lists[static_cast<int>(v.y) + lane] = key;
-          } else if (v.x != 0u) {
-            if ((v.x >> lane) & 1u) head_lists[static_cast<int>(v.y) + __popc(v.x & lt)] = key;
+          if (!dense) {                               // warp-uniform
+            if (v.x == 0xffffffffu) {
+              head_lists[static_cast<int>(v.y) + lane] = key;
+            } else if (v.x != 0u) {
+              if ((v.x >> lane) & 1u) head_lists[static_cast<int>(v.y) + __popc(v.x & lt)] = key;
+            }
           }
-          if (union_row) {                            // warp-uniform
+          if (v.w != 0xffffffffu) {                   // warp-uniform
             const uint32_t u = v.x | v.z;
             const uint32_t tag = (((v.z >> lane) & 1u) << 30) | (((v.x >> lane) & 1u) << 31);
             if (u == 0xffffffffu) {
@@ -708,7 +790,10 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
   // written even after an abort: a count never exceeds its block's capacity
   if (warp >= 2 && qtr == 0 && row_valid) {
     a.counts[(long long)bh * a.nqb + qb] = off;
-    if (paired && hs == 1) a.pair_counts[(long long)(bh0 >> 1) * a.nqb + qb] = uoff;
+    if (paired && hs == 1) {
+      a.pair_counts[(long long)(bh0 >> 1) * a.nqb + qb] = uoff;
+      a.pair_split[(long long)(bh0 >> 1) * a.nqb + qb] = split < 0 ? uoff : split;
+    }
   }
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
@@ -823,6 +908,7 @@ struct PairCompactArgs {
   long long list_per_head;
   long long cap_a;
   int* pair_counts;         // [B*Hq/2*nqb]
+  int* pair_split;          // [B*Hq/2*nqb]: union entries before the heads first differ
 };
 
 __global__ void __launch_bounds__(kCompactThreads)
@@ -867,18 +953,21 @@ pair_compact_kernel(const PairCompactArgs a) {
 
   __shared__ int warp_cnt[3][kCompactThreads / 32];
   __shared__ int warp_base[3][kCompactThreads / 32];
+  __shared__ int warp_diff[kCompactThreads / 32];
+  __shared__ int first_diff;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nw = kCompactThreads / 32;
   const int seg = (((n + nw - 1) / nw) + 31) & ~31;
   const int s_lo = w_lo + warp * seg;
   const int s_hi = min(s_lo + seg, w_hi);
-  int ca = 0, cb = 0, cu = 0;
+  int ca = 0, cb = 0, cu = 0, diff = 0x7fffffff;    // diff: first word where the heads differ
   for (int w = s_lo + lane; w < s_hi; w += 32) {
     uint32_t wa, wb;
     words_at(w, wa, wb);
     ca += __popc(wa);
     cb += __popc(wb);
     cu += __popc(wa | wb);
+    if (wa != wb) diff = min(diff, w);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
@@ -886,10 +975,13 @@ pair_compact_kernel(const PairCompactArgs a) {
     cb += __shfl_xor_sync(0xffffffffu, cb, o);
     cu += __shfl_xor_sync(0xffffffffu, cu, o);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) diff = min(diff, __shfl_xor_sync(0xffffffffu, diff, o));
   if (lane == 0) {
     warp_cnt[0][warp] = ca;
     warp_cnt[1][warp] = cb;
     warp_cnt[2][warp] = cu;
+    warp_diff[warp] = diff;
   }
   __syncthreads();
   if (threadIdx.x < 3) {
@@ -900,9 +992,16 @@ pair_compact_kernel(const PairCompactArgs a) {
     }
     if (threadIdx.x == 0) a.counts[rowA] = run;
     if (threadIdx.x == 1) a.counts[rowB] = run;
-    if (threadIdx.x == 2) a.pair_counts[row] = run;
+    if (threadIdx.x == 2) {
+      int m = 0x7fffffff;
+      for (int i = 0; i < nw; ++i) m = min(m, warp_diff[i]);
+      first_diff = m;
+      a.pair_counts[row] = run;
+      if (m == 0x7fffffff) a.pair_split[row] = run;            // the heads agree throughout
+    }
   }
   __syncthreads();
+  const int fd = first_diff;
   int base_a = warp_base[0][warp], base_b = warp_base[1][warp], base_u = warp_base[2][warp];
   const uint32_t lt = (1u << lane) - 1u;
   auto scan = [&](int v) {
@@ -930,7 +1029,10 @@ pair_compact_kernel(const PairCompactArgs a) {
       const int oa = __shfl_sync(0xffffffffu, ea, j);
       const int ob = __shfl_sync(0xffffffffu, eb, j);
       const int key = 32 * (w0 + j) + lane;
-      if ((uj >> lane) & 1u) {
+      // union entries from the first word where the heads differ (before
+      // it the union is head A's list); that word's offset is the split
+      if (w0 + j == fd && lane == 0) a.pair_split[row] = base_u + ou;
+      if (w0 + j >= fd && ((uj >> lane) & 1u)) {
         const uint32_t tag = (((aj >> lane) & 1u) << 30) | (((bj >> lane) & 1u) << 31);
         outU[base_u + ou + __popc(uj & lt)] = static_cast<uint32_t>(key) | tag;
       }
