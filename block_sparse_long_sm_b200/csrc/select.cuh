@@ -33,21 +33,23 @@ namespace spa {
 // ---------------------------------------------------------------------------
 // One CTA streams kPoolQbs consecutive query blocks of one q head: warp 0
 // loads each block's Q tile (2-stage ring) and its sink and local K tiles
-// (3-stage ring); warp 1 issues S = Q K^T per key tile into four TMEM
-// accumulators; warps 2-9 (two per TMEM lane quadrant, 64 columns each)
-// take the causal row max of every tile and, from the Q tile in shared
-// memory, the column sums of the block's rows (each warp pair half the
-// rows).  Per block the two halves are combined through shared memory
-// behind a bounded mbarrier wait: x_a = max * scale, its mean over the
-// block's rows, and avgpool(Q) * scale split into bf16 hi + lo.
+// (3-stage ring); warp 1 issues S = Q K^T per key tile into three TMEM
+// accumulators and, per block, the column sums of Q as one more MMA,
+// ones(128 x 128) * Q, into a fourth (every row of it holds the sums);
+// warps 2-9 (two per TMEM lane quadrant, 64 columns each) take the causal
+// row max of every tile.  Per block the two halves are combined through
+// shared memory behind a bounded mbarrier wait: x_a = max * scale, its mean
+// over the block's rows, and avgpool(Q) * scale split into bf16 hi + lo.  A
+// last block shorter than 128 rows sums its valid Q rows on the CUDA cores
+// instead (the tile's other rows belong to the next head).
 constexpr int kPoolQbs = 8;
 constexpr int kPoolThreads = 320;
 constexpr int kPoolQStages = 2;
 constexpr int kPoolKStages = 3;
-constexpr int kPoolBufs = 4;
+constexpr int kPoolBufs = 3;                  // S accumulators; TMEM columns [384, 512) hold the sums
 constexpr uint32_t kPoolBarBytes = 8192u;
 constexpr uint32_t kPoolSmemBytes =
-    1024u + (kPoolQStages + kPoolKStages) * kTileBytes + kPoolBarBytes;
+    1024u + (kPoolQStages + kPoolKStages + 1) * kTileBytes + kPoolBarBytes;   // + the ones tile
 static_assert(kPoolSmemBytes <= 232448u, "more shared memory than a CTA may use");
 
 struct PoolArgs {
@@ -70,7 +72,8 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t s_base = smem_u32(smem);
   auto s_q = [&](int st) { return s_base + st * kTileBytes; };
   auto s_k = [&](int st) { return s_base + (kPoolQStages + st) * kTileBytes; };
-  uint8_t* bar_area = smem + (kPoolQStages + kPoolKStages) * kTileBytes;
+  const uint32_t s_ones = s_base + (kPoolQStages + kPoolKStages) * kTileBytes;
+  uint8_t* bar_area = smem + (kPoolQStages + kPoolKStages + 1) * kTileBytes;
   const uint32_t b0 = smem_u32(bar_area);
   auto bar_qfull = [&](int s) { return b0 + 8u * s; };
   auto bar_qempty = [&](int s) { return b0 + 8u * (2 + s); };
@@ -81,10 +84,11 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
   auto bar_x = [&](int s) { return b0 + 8u * (18 + s); };       // halves combined
   auto bar_r = [&](int s) { return b0 + 8u * (20 + s); };       // row sums per quadrant
   const uint32_t bar_drain = b0 + 8u * 22;
+  const uint32_t bar_pfull = b0 + 8u * 23;                      // column sums in TMEM
+  const uint32_t bar_pfree = b0 + 8u * 24;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 256);
   volatile uint32_t* abort_flag = tmem_holder + 1;
   float* x_max = reinterpret_cast<float*>(bar_area + 512);      // [2][2 halves][128]
-  float* x_col = reinterpret_cast<float*>(bar_area + 2560);     // [2][2 halves][128]
   float* x_red = reinterpret_cast<float*>(bar_area + 4608);     // [2][4 quadrants]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -107,8 +111,10 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
   if (threadIdx.x == 0) {
     for (int s = 0; s < kPoolQStages; ++s) {
       mbar_init(bar_qfull(s), 1);
-      mbar_init(bar_qempty(s), 1 + 256);            // the MMAs' commit + every epilogue thread
+      mbar_init(bar_qempty(s), 1 + 128);            // the MMAs' commit + the q-bar threads
     }
+    mbar_init(bar_pfull, 1);
+    mbar_init(bar_pfree, 128);
     for (int s = 0; s < kPoolKStages; ++s) {
       mbar_init(bar_kfull(s), 1);
       mbar_init(bar_kempty(s), 1);
@@ -129,6 +135,12 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
+  {  // the all-ones A operand of the column-sum MMA (1.0 in bf16; any swizzle)
+    uint4* ones = reinterpret_cast<uint4*>(smem + (s_ones - s_base));
+    for (int i = threadIdx.x; i < static_cast<int>(kTileBytes / 16); i += blockDim.x)
+      ones[i] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  }
+  fence_proxy_async_smem();                         // generic-proxy writes -> tensor-core reads
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -193,7 +205,19 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit(bar_sfull(bb));
           mma_commit(bar_kempty(ks));
         }
-        if (ok) mma_commit(bar_qempty(qs));            // Q no longer read by the MMAs
+        if (!ok) break;
+        // column sums of Q: ones(128 x 128) * Q, Q read as a (rows x d) MN-major operand
+        if (i > 0 && !(ok = mbar_wait(bar_pfree, (i - 1) & 1, wc))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32u;
+          mma_bf16_ss(tmem + 384u, smem_desc_sw128(s_ones + off, 16),
+                      smem_desc_sw128(s_q(qs) + kk * 2048u, kHalfBytes), kIdescPV,
+                      kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_pfull);
+        mma_commit(bar_qempty(qs));                    // Q no longer read by the MMAs
       }
       mma_commit(bar_drain);
       mbar_drain(bar_drain, 0, a.wait_ns);
@@ -213,25 +237,26 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
       geom(qb, ls, le, sink_end, n_sink_t, T);
       const int row0 = qb * 128;
       const int nrows = le - row0;
-      // column sum of Q over this half's rows
       if (!warp_wait(bar_qfull(qs), (i / kPoolQStages) & 1, wc)) break;
-      const uint8_t* qt = smem + (s_q(qs) - s_base);
-      auto qv = [&](int rr) {
-        return __bfloat162float(
-            *reinterpret_cast<const __nv_bfloat16*>(qt + dhalf + sw128_offset(rr, dbyte)));
-      };
-      float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;   // four independent chains
-      const int r_lo = 64 * half, r_hi = min(r_lo + 64, nrows);
-      int rr = r_lo;
-      for (; rr + 4 <= r_hi; rr += 4) {
-        p0 += qv(rr);
-        p1 += qv(rr + 1);
-        p2 += qv(rr + 2);
-        p3 += qv(rr + 3);
+      // a short last block: its valid rows' column sums on the CUDA cores
+      float col_short = 0.f;
+      if (half == 1) {
+        if (nrows < 128) {
+          const uint8_t* qt = smem + (s_q(qs) - s_base);
+          float p0 = 0.f, p1 = 0.f, p2 = 0.f, p3 = 0.f;   // four independent chains
+          int rr = 0;
+          for (; rr + 4 <= nrows; rr += 4) {
+            p0 += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + dhalf + sw128_offset(rr, dbyte)));
+            p1 += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + dhalf + sw128_offset(rr + 1, dbyte)));
+            p2 += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + dhalf + sw128_offset(rr + 2, dbyte)));
+            p3 += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + dhalf + sw128_offset(rr + 3, dbyte)));
+          }
+          for (; rr < nrows; ++rr)
+            p0 += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(qt + dhalf + sw128_offset(rr, dbyte)));
+          col_short = (p0 + p1) + (p2 + p3);
+        }
+        mbar_arrive(bar_qempty(qs));
       }
-      for (; rr < r_hi; ++rr) p0 += qv(rr);
-      const float col = (p0 + p1) + (p2 + p3);
-      mbar_arrive(bar_qempty(qs));
       // causal row max over this half's columns of the block's key tiles
       float mx = -INFINITY;
       bool ok = true;
@@ -251,17 +276,23 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
         int limit = (t < n_sink_t) ? (sink_end - key0) : min(le - key0, row0 + r - key0 + 1);
         limit = max(0, min(limit, 64));
         float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        if (limit == 64) {                             // whole half tile valid
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+          for (int c = 0; c < 2; ++c)
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e < limit) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sr[c][e]));
+            for (int e = 0; e < 32; ++e) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sr[c][e]));
+        } else {
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (c * 32 + e < limit) m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(sr[c][e]));
+        }
         mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
       }
       if (!ok) break;
       // combine the two halves
       x_max[(xs * 2 + half) * 128 + r] = mx;
-      x_col[(xs * 2 + half) * 128 + r] = col;
       mbar_arrive(bar_x(xs));
       if (!warp_wait(bar_x(xs), (i >> 1) & 1, wc)) break;
       if (half == 0) {
@@ -277,8 +308,19 @@ anchor_pool_kernel(const __grid_constant__ CUtensorMap tm_q,
               (x_red[xs * 4 + 0] + x_red[xs * 4 + 1] + x_red[xs * 4 + 2] + x_red[xs * 4 + 3]) /
               static_cast<float>(nrows);
       } else {
-        // pooled query, column d = r
-        const float sum = x_col[(xs * 2) * 128 + r] + x_col[(xs * 2 + 1) * 128 + r];
+        // pooled query, column d = r: every TMEM row of the column-sum MMA holds
+        // the sums, so this thread takes column r from its own row
+        if (!warp_wait(bar_pfull, i & 1, wc)) break;
+        tc_fence_after();
+        uint32_t cs[32];
+        tmem_ld32(tmem + lane_off + 384u + 32u * quad, cs);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(bar_pfree);
+        float sum = 0.f;
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sum = e == lane ? __uint_as_float(cs[e]) : sum;
+        if (nrows < 128) sum = col_short;
         const float qbar = (sum / static_cast<float>(nrows)) * a.scale;
         const __nv_bfloat16 hi = __float2bfloat16_rn(qbar);
         const __nv_bfloat16 lo = __float2bfloat16_rn(qbar - __bfloat162float(hi));
