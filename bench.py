@@ -113,7 +113,7 @@ class ClockSampler:
 def _kernel_source_hash() -> str:
     import hashlib
     h = hashlib.sha256()
-    for name in ("attn.cuh", "attn_pair.cuh", "ptx.cuh"):
+    for name in ("attn.cuh", "attn_pair.cuh", "common.cuh", "ptx.cuh"):
         with open(os.path.join(ROOT, "block_sparse_long_sm_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()
