@@ -222,8 +222,14 @@ def main():
     ap.add_argument("--theta", type=float, default=5.0)
     ap.add_argument("--config", default=C2_LLAMA_128K.name, choices=sorted(CONFIGS))
     ap.add_argument("--no-extras", action="store_true", help="skip SALE/dense/e2e/cpu legs")
+    ap.add_argument("--sweep", action="store_true",
+                    help="density sweep instead of the headline step: one JSON line per "
+                         "(layer, theta), theta from +inf to 2, with the same kernel run dense")
     args = ap.parse_args()
     w = CONFIGS[args.config]
+    if args.sweep:
+        sweep()
+        return
     if args.impl == "reference":
         run_reference(args, w)
         return
@@ -328,6 +334,77 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def sweep():
+    """Kept fraction vs time and vs tensor peak over theta (the density sweep
+    of the 128K Llama layer, its B = 4, L = 16384 variant and the 64K Qwen
+    layer with half its kv heads diffuse).  One JSON line per point; theta =
+    +inf is compared with DENSE mode (same kernel, every causal key)."""
+    import torch
+    import block_sparse_long_sm_b200 as spa
+    from workloads import C3_QWEN_64K, C4_B4_16K, C4_SWEEP_128K, THETA_DENSITY_SWEEP
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    peaks = _peaks()
+
+    def timed(fn, reps=3, warm=2):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    plan = [(C4_SWEEP_128K, THETA_DENSITY_SWEEP), (C4_B4_16K, THETA_DENSITY_SWEEP),
+            (C3_QWEN_64K, (5.0,))]
+    for w, thetas in plan:
+        inp = generate(w)
+        to = lambda u: torch.from_numpy(np.ascontiguousarray(u).view(np.int16)).to(dev).view(torch.bfloat16)
+        q, k, v = to(inp.q), to(inp.k), to(inp.v)
+        del inp
+        B, Hq, Hkv, L = w.batch, w.heads_q, w.heads_kv, w.seq_len
+        o = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
+        pd = spa.make_params(B, Hq, Hkv, L, mode="dense", sink=w.sink, local=w.local)
+        wsd = torch.empty(spa.sparse_prefill_workspace_bytes(pd), dtype=torch.uint8, device=dev)
+        spa.check(spa.sparse_prefill_plan(pd, q, k, wsd, stream=stream))
+        dense_ms = timed(lambda: spa.check(spa.sparse_prefill_attn(pd, q, k, v, wsd, o, None,
+                                                                   stream=stream)))
+        st, sd = spa.sparse_prefill_stats(pd, wsd, stream=stream)
+        spa.check(st, "stats")
+        del wsd
+        for theta in thetas:
+            p = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=w.sink, local=w.local,
+                                theta=theta)
+            ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
+            plan_ms = timed(lambda: spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream)))
+            attn_ms = timed(lambda: spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None,
+                                                                      stream=stream)))
+            st, s = spa.sparse_prefill_stats(p, ws, stream=stream)
+            spa.check(st, "stats")
+            flops = spa.kept_flops(s)
+            alg_bytes = 2 * B * Hq * L * 128 + 2 * B * Hkv * L * 128 + 4 * s.kept_candidates
+            print(json.dumps({
+                "sweep": "density", "workload": w.name, "theta": theta,
+                "kept_fraction": s.kept_pairs / s.dense_pairs,
+                "kept_candidates_fraction": s.kept_candidates / max(1, s.candidates),
+                "plan_ms": plan_ms, "attn_ms": attn_ms, "step_ms": plan_ms + attn_ms,
+                "attn_tflops": flops / (attn_ms / 1e3) / 1e12,
+                "attn_frac": flops / (attn_ms / 1e3) / 1e12 / peaks["bf16_sus"],
+                "selection_gbs": alg_bytes / (plan_ms / 1e3) / 1e9,
+                "selection_frac": alg_bytes / (plan_ms / 1e3) / 1e9 / peaks["hbm"],
+                "dense_attn_ms": dense_ms, "speedup_vs_dense": dense_ms / (plan_ms + attn_ms),
+                "peak_source": peaks["src"]}), flush=True)
+            del ws
+        del q, k, v, o
+        torch.cuda.empty_cache()
 
 
 def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, stats):
