@@ -794,13 +794,38 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) hl[__shfl_sync(0xffffffffu, pos, j)] = key;
       }
-      if (!dense || __any_sync(0xffffffffu, write_union)) {
+      // rows with something to store: own keys (unless stored above) or union entries
+      const uint32_t need = __ballot_sync(
+          0xffffffffu, (!dense && w != 0u) || (write_union && (w | awq) != 0u));
+      // few keys per row (every word of the warp at most 8 bits): each thread
+      // stores its own row's keys, one per step, instead of a warp-wide store
+      // per row
+      const uint32_t uw = write_union ? (w | awq) : 0u;
+      const bool sparse = need != 0u &&
+          __reduce_max_sync(0xffffffffu, max(dense ? 0 : __popc(w), __popc(uw))) <= 8;
+      if (sparse) {
+        uint32_t rem = dense ? 0u : w, urem = uw;
+        int k = 0, ku = 0;
+        const int upos = row_elem + uoff + ubefore;
+        while (__any_sync(0xffffffffu, (rem | urem) != 0u)) {
+          if (rem) {
+            head_lists[pos + k++] = key0 + __ffs(rem) - 1;
+            rem &= rem - 1u;
+          }
+          if (urem) {
+            const int e = __ffs(urem) - 1;
+            const uint32_t tag = (((awq >> e) & 1u) << 30) | (((w >> e) & 1u) << 31);
+            pair_list[upos + ku++] = static_cast<uint32_t>(key0 + e) | tag;
+            urem &= urem - 1u;
+          }
+        }
+      } else if (need) {
         my_stage[lane] = make_uint4(w, static_cast<uint32_t>(pos), awq,
                                     write_union ? static_cast<uint32_t>(row_elem + uoff + ubefore)
                                                 : 0xffffffffu);
         __syncwarp();
-#pragma unroll 4
-        for (int j = 0; j < 32; ++j) {
+        for (uint32_t rows = need; rows; rows &= rows - 1u) {
+          const int j = __ffs(rows) - 1;
           const uint4 v = my_stage[j];
           if (!dense) {                               // warp-uniform
             if (v.x == 0xffffffffu) {
