@@ -303,7 +303,9 @@ def main():
     attn_avg = sum(attn_ms) / len(attn_ms)
     achieved = flops_step / (attn_avg / 1e3) / 1e12
     extras = {}
-    n_launch_plan = {"anchor": 3, "sale": 6, "dense": 0}[args.mode]
+    # kernels per plan: anchor = pooling + fused scan/compaction (the bench uses
+    # step 1); SALE = two K-mean passes, two quantisations, scan, compaction
+    n_launch_plan = {"anchor": 2, "sale": 6, "dense": 0}[args.mode]
     launches = (n_launch_plan + 1) * args.steps
 
     if rank == 0 and not args.no_extras:
