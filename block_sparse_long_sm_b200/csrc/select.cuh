@@ -534,22 +534,25 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 // share the kv head, so each K tile feeds both).  The CTA walks every key tile
 // of its candidate range in ascending order and appends each query block's
 // kept keys to the block's list at a running offset, so the lists come out
-// ascending with no intermediate mask.  For a pair it also writes the union
-// of the two heads' kept keys per query block, each entry tagged with the
-// heads that kept it (index | in 2p << 30 | in 2p+1 << 31), and its size:
-// the paired attention kernel's key list.  Selection groups (step > 1) must
-// lie inside one warp: step a power of two <= 32.
+// ascending with no intermediate mask.  For a pair it also builds the union
+// of the two heads' kept keys per query block (the paired attention kernel's
+// key list): its size, the number of its entries before the two heads'
+// selections first differ (up to there the union is head 2p's own list),
+// and, from that point on, the entries themselves, each tagged with the heads
+// that kept it (index | in 2p << 30 | in 2p+1 << 31).  Selection groups
+// (step > 1) must lie inside one warp: step a power of two <= 32.
 //
 // Warp 0 loads the pooled-Q tile once and the K tiles (4-stage ring); warp 1
 // issues the hi and lo MMAs into four TMEM accumulators; warps 2-17 each own
 // a TMEM lane quadrant and 32 of the 128 columns (one 32-key word per row).
 // Per key tile the sixteen warps exchange their words through shared memory
 // behind a bounded mbarrier wait, so that every thread knows its row's kept
-// count before its word; each warp then stages its rows' (word, list
-// position) pairs and writes the kept keys with one coalesced store per row
-// (a single add per row when all 32 keys are kept).  CTAs are numbered
-// heaviest first (last M tile first), so the block scheduler fills the GPU
-// longest-job-first.
+// count before its word.  Stores, by density of the warp's 32 words: all keys
+// kept -- one shuffle and one coalesced store of the same 32 values per row;
+// at most 8 keys in every word -- each thread stores its own row's keys; in
+// between -- the rows' (word, list position) pairs are staged and each row
+// with keys is one coalesced store.  CTAs are numbered heaviest first (last M
+// tile first), so the block scheduler fills the GPU longest-job-first.
 constexpr int kSelEpiWarps = 16;
 constexpr int kSelThreads = 32 * (2 + kSelEpiWarps);
 constexpr int kSelStages = 4;
