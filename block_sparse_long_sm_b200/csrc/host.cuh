@@ -125,8 +125,9 @@ Layout layout_of(const spa_params* p) {
   }
   lo.paired = (lo.group % 2) == 0;
   if (lo.paired && p->mode != SPA_MODE_DENSE) {
-    // tagged union lists of head pairs and their sizes, for the paired
-    // attention kernel (opaque scratch)
+    // for the paired attention kernel (opaque scratch): per (b, head pair,
+    // query block) the union size, the split (union entries shared with head
+    // 2p's list) and the tagged union entries from the split on
     lo.pair_counts = take((lo.nb / 2) * 4);
     lo.pair_split = take((lo.nb / 2) * 4);
     lo.pair_lists = take((size_t)(bh / 2) * lo.list_per_head * 4);

@@ -140,7 +140,8 @@ SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   }
   if (lo.paired) {
-    // one pass writes both heads' lists and their tagged union list
+    // one pass writes both heads' lists, their union's size and split, and
+    // the tagged union entries from the first difference on
     PairCompactArgs pc{lo.nqb, Hq, p->sink, p->local, lo.unit, p->step,
                        reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
                        reinterpret_cast<int*>(ws + lo.lists), reinterpret_cast<int*>(ws + lo.counts),
