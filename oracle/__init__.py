@@ -27,11 +27,16 @@ Modules:
 
 * ``selection`` -- anchor (stripe) selection and SALE (block) selection;
 * ``attention`` -- masked softmax attention over a kept key set, and an
-  independently written dense causal attention.
+  independently written dense causal attention;
+* ``calibration`` -- SALE's per-head tau calibration (Sec. 3.3, Appendix C);
+* ``decode`` -- decode-shaped reuse of a prefill plan (SpotAttention Fig. 2,
+  Sec. 3; KVpop Sec. 3, transposed attention);
+* ``fp8`` -- E4M3 rounding and SageAttention-style quantisation for an FP8
+  Computation Pass (SALE review, Summary).
 
 Every function here is pinned by tests in ``tests/test_oracle_*.py`` against
 closed forms, invariants, special cases and brute force; see the module
 docstrings for which pin covers which function.
 """
 
-from . import attention, selection  # noqa: F401
+from . import attention, calibration, decode, fp8, selection  # noqa: F401
