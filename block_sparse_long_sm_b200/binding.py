@@ -24,7 +24,8 @@ SPA_DEBUG_STALL_ATTN = 0x1
 MODES = {"anchor": SPA_MODE_ANCHOR, "sale": SPA_MODE_SALE, "dense": SPA_MODE_DENSE}
 
 EXPORTED = ("sparse_prefill_workspace_bytes", "sparse_prefill_plan", "sparse_prefill_attn",
-            "sparse_prefill_stats", "sparse_prefill_status_string")
+            "sparse_prefill_stats", "sparse_prefill_status_string", "sparse_prefill_plan_static",
+            "sparse_decode_scratch_bytes", "sparse_decode_prepare", "sparse_decode_attn")
 
 
 class SpaParams(ctypes.Structure):
@@ -75,6 +76,13 @@ def _load():
     lib.sparse_prefill_stats.restype = ctypes.c_int
     lib.sparse_prefill_plan_static.argtypes = [P, vp, vp, vp, vp, sz, vp, vp]
     lib.sparse_prefill_plan_static.restype = ctypes.c_int
+    i32 = ctypes.c_int32
+    lib.sparse_decode_scratch_bytes.argtypes = [P, i32]
+    lib.sparse_decode_scratch_bytes.restype = sz
+    lib.sparse_decode_prepare.argtypes = [P, i32, vp, sz, vp, sz, vp]
+    lib.sparse_decode_prepare.restype = ctypes.c_int
+    lib.sparse_decode_attn.argtypes = [P, vp, vp, vp, i32, i32, vp, sz, vp, sz, vp, vp, vp]
+    lib.sparse_decode_attn.restype = ctypes.c_int
     lib.sparse_prefill_status_string.argtypes = [ctypes.c_int]
     lib.sparse_prefill_status_string.restype = ctypes.c_char_p
     return lib
@@ -162,6 +170,30 @@ def sparse_prefill_plan_static(params: SpaParams, q, k, counts, lists, lists_ele
     return int(_lib.sparse_prefill_plan_static(ctypes.byref(params), _ptr(q), _ptr(k),
                                                _ptr(counts), _ptr(lists), n, _ptr(error_word),
                                                _stream(stream)))
+
+
+def sparse_decode_scratch_bytes(params: SpaParams, kv_capacity: int) -> int:
+    return int(_lib.sparse_decode_scratch_bytes(ctypes.byref(params), int(kv_capacity)))
+
+
+def sparse_decode_prepare(params: SpaParams, kv_capacity: int, workspace, scratch,
+                          workspace_bytes=None, scratch_bytes=None, stream=None) -> int:
+    """Once per plan: the tagged union of each kv head's q-head selections."""
+    wb = _nbytes(workspace) if workspace_bytes is None else int(workspace_bytes)
+    sb = _nbytes(scratch) if scratch_bytes is None else int(scratch_bytes)
+    return int(_lib.sparse_decode_prepare(ctypes.byref(params), int(kv_capacity), _ptr(workspace),
+                                          wb, _ptr(scratch), sb, _stream(stream)))
+
+
+def sparse_decode_attn(params: SpaParams, q, k_cache, v_cache, kv_capacity: int, pos: int,
+                       workspace, scratch, o, lse=None, workspace_bytes=None,
+                       scratch_bytes=None, stream=None) -> int:
+    """One decoding query per (b, q head) at position ``pos`` over sink + selection + window."""
+    wb = _nbytes(workspace) if workspace_bytes is None else int(workspace_bytes)
+    sb = _nbytes(scratch) if scratch_bytes is None else int(scratch_bytes)
+    return int(_lib.sparse_decode_attn(ctypes.byref(params), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                       int(kv_capacity), int(pos), _ptr(workspace), wb,
+                                       _ptr(scratch), sb, _ptr(o), _ptr(lse), _stream(stream)))
 
 
 def sparse_prefill_status_string(status: int) -> str:

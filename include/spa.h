@@ -209,6 +209,46 @@ SPA_API spa_status sparse_prefill_plan_static(const spa_params* p, const void* q
                                               size_t lists_elems, uint32_t* error_word,
                                               cudaStream_t stream);
 
+/* Decode-shaped reuse of a finished plan (SpotAttention, Fig. 2 and Sec. 3:
+ * a decoding query attends to a sink prefix, a recency window and a set of
+ * selected blocks).  The selected part is the plan's selection for the last
+ * prompt query block qb = (L - 1) / 128, so one query per (b, q head) at
+ * absolute position pos (L - 1 <= pos < kv_capacity, the same for every
+ * sequence) attends to
+ *
+ *   D_h(pos) = [0, min(sink, pos + 1)) u sel_h(qb) u [max(ls_qb, min(sink, pos + 1)), pos],
+ *
+ * every key up to pos in DENSE mode.  At pos = L - 1 this is the key set the
+ * prefill gave its last prompt row.  p is the plan's params (seq_len = L, the
+ * prompt length); the workspace is the plan's and is only read, except for
+ * its error word.
+ *
+ *   scratch      caller-owned device buffer of sparse_decode_scratch_bytes
+ *                (16-byte aligned) shared by prepare and attn: the union of
+ *                each kv head's q heads' selections and the split partials;
+ *   kv_capacity  rows per (b, kv head) of the K/V cache, L <= kv_capacity <= 2^24;
+ *   q            bf16 [B, Hq, 128], the decoding queries;
+ *   k_cache, v_cache  bf16 [B, Hkv, kv_capacity, 128]; rows 0..pos must hold
+ *                the keys/values of positions 0..pos (the prompt's at 0..L-1);
+ *   o            bf16 [B, Hq, 128]; lse: optional fp32 [B, Hq] (natural log).
+ *
+ * sparse_decode_prepare runs once per plan (it merges the selections of the
+ * q heads of each kv head into one list with per-head bits); every
+ * sparse_decode_attn call after it, at any pos, reuses that list until the
+ * next plan or prepare on the same buffers.  Argument errors are returned
+ * before any launch; a list entry outside its block's candidates sets the
+ * bad-index bit of the workspace error word (reported by
+ * sparse_prefill_stats). */
+SPA_API size_t sparse_decode_scratch_bytes(const spa_params* p, int32_t kv_capacity);
+SPA_API spa_status sparse_decode_prepare(const spa_params* p, int32_t kv_capacity,
+                                         void* workspace, size_t workspace_bytes, void* scratch,
+                                         size_t scratch_bytes, cudaStream_t stream);
+SPA_API spa_status sparse_decode_attn(const spa_params* p, const void* q, const void* k_cache,
+                                      const void* v_cache, int32_t kv_capacity, int32_t pos,
+                                      void* workspace, size_t workspace_bytes, void* scratch,
+                                      size_t scratch_bytes, void* o, float* lse,
+                                      cudaStream_t stream);
+
 /* Static string for a status code. */
 SPA_API const char* sparse_prefill_status_string(spa_status s);
 

@@ -10,6 +10,8 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (sm_100a) and the built library")
+    config.addinivalue_line("markers", "gpu_pending: GPU test not yet run on a B200; "
+                            "joins the gpu set after its first passing run")
     config.addinivalue_line("markers", "slow: long-running CPU check")
 
 
@@ -23,5 +25,5 @@ def pytest_collection_modifyitems(config, items):
         return
     skip = pytest.mark.skip(reason="no CUDA device")
     for item in items:
-        if "gpu" in item.keywords:
+        if "gpu" in item.keywords or "gpu_pending" in item.keywords:
             item.add_marker(skip)

@@ -101,3 +101,48 @@ def test_shard_units_partition():
             seen += shard_units(B, H, world, r)
         assert seen == [(b, g) for b in range(B) for g in range(H)]
     assert kv_head_slice(8, 2, 1) == (4, 8)
+
+
+def test_decode_scratch_bytes():
+    p = spa.make_params(1, 32, 8, 131072)
+    n = spa.sparse_decode_scratch_bytes(p, 131072 + 1024)
+    # union of each kv head's selections (4 B per candidate), its tag words
+    # (1 B per candidate) and the split partials: a few MB, independent of pos
+    cand = 131072 - 256 - 128
+    assert 8 * cand * 5 < n < 8 * cand * 5 + 4e6
+    assert spa.sparse_decode_scratch_bytes(p, 131072) <= n
+    assert spa.sparse_decode_scratch_bytes(p, 131071) == 0          # capacity below L
+    assert spa.sparse_decode_scratch_bytes(p, (1 << 24) + 1) == 0   # beyond 2^24 rows
+    assert spa.sparse_decode_scratch_bytes(spa.make_params(1, 4, 2, 0), 16) == 0
+    assert spa.sparse_decode_scratch_bytes(spa.make_params(1, 4, 2, 100, head_dim=64), 128) == 0
+    for mode, bk in (("anchor", None), ("sale", 32), ("dense", None)):
+        for hq, hkv in ((4, 2), (6, 2), (16, 1), (24, 1)):
+            assert spa.sparse_decode_scratch_bytes(
+                spa.make_params(2, hq, hkv, 3000, mode=mode, block_k=bk), 4000) > 0
+
+
+def test_decode_validation_before_any_launch():
+    p = spa.make_params(1, 4, 2, 1024, sink=64, local=128)
+    ws = spa.sparse_prefill_workspace_bytes(p)
+    sc = spa.sparse_decode_scratch_bytes(p, 1100)
+    A, S, Q = 1 << 20, 1 << 24, 1 << 28          # aligned stand-in addresses, never touched
+
+    def attn(pos, cap=1100, ws_bytes=ws, sc_bytes=sc, scratch=S):
+        return spa.sparse_decode_attn(p, Q, Q, Q, cap, pos, A, scratch, Q, None,
+                                      workspace_bytes=ws_bytes, scratch_bytes=sc_bytes, stream=0)
+    assert attn(1022) == spa.SPA_ERR_INVALID            # pos < L - 1
+    assert attn(1100) == spa.SPA_ERR_INVALID            # pos >= capacity
+    assert attn(1023, cap=1000) == spa.SPA_ERR_INVALID  # capacity < L
+    assert attn(1023, cap=(1 << 24) + 1) == spa.SPA_ERR_UNSUPPORTED
+    assert attn(1023, sc_bytes=sc - 1) == spa.SPA_ERR_WORKSPACE
+    assert attn(1023, ws_bytes=ws - 1) == spa.SPA_ERR_WORKSPACE
+    assert attn(1023, scratch=S + 8) == spa.SPA_ERR_INVALID
+    assert spa.sparse_decode_attn(p, 0, Q, Q, 1100, 1023, A, S, Q, None, workspace_bytes=ws,
+                                  scratch_bytes=sc, stream=0) == spa.SPA_ERR_INVALID
+    assert spa.sparse_decode_prepare(p, 1100, A, S, workspace_bytes=ws, scratch_bytes=sc - 1,
+                                     stream=0) == spa.SPA_ERR_WORKSPACE
+    assert spa.sparse_decode_prepare(p, 1100, 0, S, workspace_bytes=ws, scratch_bytes=sc,
+                                     stream=0) == spa.SPA_ERR_INVALID
+    bad = spa.make_params(1, 4, 2, 1024, sink=64, local=100)
+    assert spa.sparse_decode_prepare(bad, 1100, A, S, workspace_bytes=ws, scratch_bytes=sc,
+                                     stream=0) == spa.SPA_ERR_INVALID
