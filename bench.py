@@ -19,6 +19,8 @@ layer (independent problems, weak scaling, no collective on the data path);
 the timed region is bracketed by barriers and the max over ranks is reported.
 
 ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
+``--sweep`` runs the density sweep and ``--decode`` the decode steps that
+reuse a plan; each prints its own JSON lines instead of the headline step.
 """
 
 from __future__ import annotations
@@ -225,10 +227,16 @@ def main():
     ap.add_argument("--sweep", action="store_true",
                     help="density sweep instead of the headline step: one JSON line per "
                          "(layer, theta), theta from +inf to 2, with the same kernel run dense")
+    ap.add_argument("--decode", action="store_true",
+                    help="decode-shaped reuse of the plan instead of the headline step: one "
+                         "decoding query per q head per step at positions L-1, L, ...")
     args = ap.parse_args()
     w = CONFIGS[args.config]
     if args.sweep:
         sweep()
+        return
+    if args.decode:
+        decode_bench(args, w)
         return
     if args.impl == "reference":
         run_reference(args, w)
@@ -407,6 +415,114 @@ def sweep():
             del ws
         del q, k, v, o
         torch.cuda.empty_cache()
+
+
+def decode_bench(args, w: Workload):
+    """Decode steps that reuse one plan: after sparse_prefill_plan (untimed) and
+    sparse_decode_prepare, step t runs sparse_decode_attn for one query per
+    q head at position L - 1 + t against a K/V cache of L + steps + 64 rows.
+    Every step reads about 0.5 GB of K/V at the 128K layer (more than L2), so
+    no flush is needed.  The roofline counts 512 bytes per key of each kv
+    head's key set (sink + union of its q heads' selections + window) plus q
+    and O, over the time of the whole call (both kernels)."""
+    import torch
+    import block_sparse_long_sm_b200 as spa
+    world, rank, local = _dist()
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    inp = generate(w)
+    B, Hq, Hkv, L = w.batch, w.heads_q, w.heads_kv, w.seq_len
+    n_steps = max(3, args.warmup) + args.steps
+    cap = L + n_steps + 64
+    to = lambda u: torch.from_numpy(np.ascontiguousarray(u).view(np.int16)).to(dev).view(torch.bfloat16)
+    q, k = to(inp.q), to(inp.k)
+    k_cache = torch.empty((B, Hkv, cap, 128), dtype=torch.bfloat16, device=dev)
+    v_cache = torch.empty((B, Hkv, cap, 128), dtype=torch.bfloat16, device=dev)
+    k_cache[:, :, :L] = k
+    v_cache[:, :, :L] = to(inp.v)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234)
+    k_cache[:, :, L:] = torch.randn((B, Hkv, cap - L, 128), generator=g, device=dev).to(torch.bfloat16)
+    v_cache[:, :, L:] = torch.randn((B, Hkv, cap - L, 128), generator=g, device=dev).to(torch.bfloat16)
+    del inp
+    p = spa.make_params(B, Hq, Hkv, L, mode=args.mode, sink=w.sink, local=w.local,
+                        theta=args.theta, tau=w.tau,
+                        block_k=w.block_k if args.mode == "sale" else None)
+    ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
+    spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream), "plan")
+    del q, k
+    sc = torch.empty(spa.sparse_decode_scratch_bytes(p, cap), dtype=torch.uint8, device=dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    spa.check(spa.sparse_decode_prepare(p, cap, ws, sc, stream=stream), "prepare")
+    b.record(stream)
+    torch.cuda.synchronize()
+    prepare_ms = a.elapsed_time(b)
+    qd = torch.randn((B, Hq, 128), generator=g, device=dev).to(torch.bfloat16)
+    od = torch.empty((B, Hq, 128), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+
+    def call(pos):
+        spa.check(spa.sparse_decode_attn(p, qd, k_cache, v_cache, cap, pos, ws, sc, od, lse,
+                                         stream=stream), "decode")
+
+    warm = max(3, args.warmup)
+    for t in range(warm):
+        call(L - 1 + t)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            call(L - 1 + warm + i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    ms = [x.elapsed_time(y) for x, y in ev]
+    st, _ = spa.sparse_prefill_stats(p, ws, stream=stream)
+    spa.check(st, "stats")
+
+    # key-set sizes per (b, kv head, subgroup) from the prepared union counts
+    group = Hq // Hkv
+    gh = next(d for d in range(8, 0, -1) if group % d == 0)
+    units = B * Hkv * (group // gh)
+    counts = sc[:4 * units].view(torch.int32).cpu().numpy().astype(np.int64)
+    qb = (L - 1) // 128
+    ls = max(0, (qb + 1) * 128 - w.local)
+    uk = w.block_k if args.mode == "sale" else 1
+    bytes_steps = []
+    for i in range(args.steps):
+        pos = L - 1 + warm + i
+        if args.mode == "dense":
+            keys = units * (pos + 1)
+        else:
+            s1 = min(w.sink, pos + 1)
+            keys = int(np.sum(s1 + counts * uk + (pos + 1 - max(ls, s1))))
+        bytes_steps.append(512 * keys + 2 * 2 * 128 * B * Hq)
+    peaks = _peaks()
+    ms_med = statistics.median(ms)
+    alg = statistics.median(bytes_steps)
+    gbs = alg / (ms_med / 1e3) / 1e9
+    line = {
+        "metric": "decode step reusing the prefill plan (one query per q head)",
+        "value": 1e3 / ms_med * B, "unit": "decoded tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": warm, "ms_per_step": ms_med, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(_config(w, args), kv_capacity=cap, prepare_ms=prepare_ms,
+                       l2="K/V read per step larger than L2 (126 MB); no flush"),
+        "roofline": {"bound": "hbm", "kernel": "decode_attn_kernel (+ decode_combine_kernel)",
+                     "achieved": gbs, "peak": peaks["hbm"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm"], "traffic": None,
+                     "algorithmic_bytes": alg,
+                     "peak_source": f"{peaks['src']} HBM copy bandwidth"},
+        "clocks": clk.summary(),
+        "gpu_launches": 2 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
 
 
 def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, stats):
