@@ -7,7 +7,12 @@
 * a block's largest magnitude quantises to +-448; data already on the E4M3
   grid at a power-of-two scale quantises exactly;
 * the K smoothing shifts every score of a row by one constant, so the
-  softmax over the smoothed keys equals the softmax over the raw keys.
+  softmax over the smoothed keys equals the softmax over the raw keys, and
+  the quantised K of grid-valued keys does not change when one vector is
+  added to every key;
+* every dequantised Q, K and V element is within half an E4M3 step of its
+  input at its group's scale (2^-4 relative, or s * 2^-10 on the subnormal
+  range).
 """
 
 import numpy as np
@@ -78,3 +83,35 @@ def test_smoothing_leaves_the_softmax_unchanged():
     b = softmax(q.astype(np.float64) @ ks.astype(np.float64).T)
     assert np.allclose(a, b, atol=1e-9)
     assert np.all(np.abs(ks.astype(np.float64).mean(axis=0)) < 1e-4)
+
+
+def test_quantised_k_is_invariant_to_a_common_key_shift():
+    # keys on a 1/8 grid with a grid-valued shift: the fp32 mean and the
+    # subtraction are exact, so smoothing removes the shift exactly
+    rng = np.random.default_rng(3)
+    k = (rng.integers(-40, 41, size=(64, 32)) / 8.0).astype(np.float32)
+    c = (rng.integers(-16, 17, size=32) / 4.0).astype(np.float32)
+    c0, s0 = fp8.quantize_k(k)
+    c1, s1 = fp8.quantize_k(k + c)
+    assert s0 == s1 and np.array_equal(c0, c1)
+
+
+def test_dequantised_operands_within_half_a_step():
+    # |x - x^| <= half an E4M3 step at x / s: 2^-4 |x| on the normal range,
+    # s * 2^-10 on the subnormal range; nothing saturates since |x| / s <= 448
+    rng = np.random.default_rng(4)
+    q = (rng.standard_normal((300, 128)) * rng.choice([0.01, 1.0, 30.0], (300, 1))).astype(np.float32)
+    k = (rng.standard_normal((300, 128)) + 2.0).astype(np.float32)
+    v = (rng.standard_normal((300, 128)) * rng.choice([0.1, 5.0], (1, 128))).astype(np.float32)
+    q_hat, k_hat, v_hat = fp8.dequantized_head(q, k, v)
+    _, qs = fp8.quantize_q(q)
+    _, ks = fp8.quantize_k(k)
+    _, vs = fp8.quantize_v(v)
+    s_q = np.repeat(qs.astype(np.float64), 128)[:300, None]
+    ksm = fp8.smooth_k(k).astype(np.float64)
+    for x, xh, s in ((q.astype(np.float64), q_hat, s_q), (ksm, k_hat, np.float64(ks)),
+                     (v.astype(np.float64), v_hat, vs.astype(np.float64)[None, :])):
+        bound = np.maximum(2.0 ** -4 * np.abs(x), s * 2.0 ** -10) * (1 + 1e-6)
+        assert np.all(np.abs(x - xh) <= bound)
+        # the largest magnitude of each scaling group maps to exactly 448
+    assert np.max(np.abs(q_hat[:128])) == np.float64(qs[0]) * 448.0
