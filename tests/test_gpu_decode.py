@@ -5,7 +5,12 @@ selection for the last prompt query block and that block's local window grown
 up to pos.  As in the prefill output tests, the selection the GPU used is
 first checked against the oracle (bit-exact up to near-ties), then the
 outputs are compared with the oracle's decode attention over the GPU's own
-kept set: max |dO| <= 1e-2, mean <= 1e-3, |dLSE| <= 2e-3 against fp64.
+kept set against fp64: |dLSE| <= 2e-3 always; on key sets of at least 128
+keys max |dO| <= 1e-2 and mean <= 1e-3; on smaller key sets, where O is not
+an average of many rows and its rounding to bf16 alone can exceed a mean of
+1e-3 (half an ulp is 0.0078 at |O| in [2, 4)), every element obeys the bound
+of the kernel's arithmetic, |dO| <= 2^-8 |O| + 1e-4 (the kernel keeps the
+probabilities in fp32 and rounds only O).
 
 Cases: GQA groups of 2, 3, 4 and 16 q heads (one to eight heads per CTA, two
 head subgroups), ANCHOR, SALE and DENSE, positions from L - 1 (where the
@@ -13,8 +18,9 @@ decode key set is the last prompt row's prefill key set) to the end of the
 cache, a prompt of one token, a sink that covers the whole candidate range,
 repeated calls after one prepare, and the 128K Llama layer.
 
-These tests carry the ``gpu_pending`` marker until their first run on a
-B200; ``pytest -m gpu_pending`` selects them.
+Tests marked ``gpu_pending`` have not yet passed on a B200 and join the
+``gpu`` set after their first passing run (``pytest -m gpu_pending`` selects
+them).
 """
 
 import numpy as np
@@ -28,7 +34,7 @@ from workloads import C0_TINY, C2_LLAMA_128K, bf16_bits_to_f32, generate, random
 from gpu_common import (LSE_ABS, O_MAX_ABS, O_MEAN_ABS, Run, compare_anchor_masks,
                         compare_sale_masks, head_f64, to_dev)
 
-pytestmark = pytest.mark.gpu_pending
+SMALL_SET = 128      # key sets below this size get the element-wise bound
 
 
 class Decode:
@@ -79,13 +85,19 @@ class Decode:
                                         sink=p.sink, local=p.local)
             qv = bf16_bits_to_f32(q_u16[b, h]).astype(np.float64)
             o_ref, lse_ref = odec.decode_attend(qv, kh, vh, keys)
-            errs.append(np.abs(o[b, h] - o_ref))
+            d = np.abs(o[b, h] - o_ref)
+            if keys.size >= SMALL_SET:
+                errs.append(d)
+            else:
+                lim = 2.0 ** -8 * np.abs(o_ref) + 1e-4
+                assert np.all(d <= lim), (b, h, pos, int(keys.size), float(np.max(d / lim)))
             lse_err = max(lse_err, abs(float(lse[b, h]) - lse_ref))
-        e = np.concatenate(errs)
-        res = dict(max_abs=float(e.max()), mean_abs=float(e.mean()), lse_max=lse_err)
-        assert res["max_abs"] <= O_MAX_ABS, res
-        assert res["mean_abs"] <= O_MEAN_ABS, res
-        assert res["lse_max"] <= LSE_ABS, res
+        assert lse_err <= LSE_ABS, lse_err
+        if errs:
+            e = np.concatenate(errs)
+            res = dict(max_abs=float(e.max()), mean_abs=float(e.mean()), lse_max=lse_err)
+            assert res["max_abs"] <= O_MAX_ABS, res
+            assert res["mean_abs"] <= O_MEAN_ABS, res
         return o, lse
 
 
@@ -93,6 +105,7 @@ def _queries(B, Hq, seed, bias=0.0):
     return random_bf16((B, Hq, 128), seed, mean=bias)
 
 
+@pytest.mark.gpu
 @pytest.mark.parametrize("hq,hkv,theta", [(4, 2, 2.5), (6, 2, 3.0), (4, 1, 2.0), (16, 1, 2.5)])
 def test_anchor_groups_and_positions(hq, hkv, theta):
     L, cap = 2000, 2100
@@ -106,6 +119,7 @@ def test_anchor_groups_and_positions(hq, hkv, theta):
         dec.compare(_queries(1, hq, 100 + i, bias=0.5), pos)
 
 
+@pytest.mark.gpu
 def test_last_prompt_row_matches_prefill():
     L, cap = 1500, 1600
     w = C0_TINY.with_(heads_q=4, heads_kv=2, sink=64, local=256)
@@ -121,6 +135,7 @@ def test_last_prompt_row_matches_prefill():
     assert np.max(np.abs(lse - lse_pre)) <= 2 * LSE_ABS
 
 
+@pytest.mark.gpu
 @pytest.mark.parametrize("bk,tau", [(64, 1e-2), (32, 1e-3)])
 def test_sale_blocks(bk, tau):
     L, cap = 1500, 1536
@@ -134,6 +149,7 @@ def test_sale_blocks(bk, tau):
         dec.compare(_queries(1, 2, 200 + i), pos)
 
 
+@pytest.mark.gpu
 def test_dense_mode():
     L, cap = 700, 800
     w = C0_TINY.with_(heads_q=4, heads_kv=2)
@@ -144,6 +160,7 @@ def test_dense_mode():
     dec.compare(_queries(1, 4, 301), cap - 1)
 
 
+@pytest.mark.gpu_pending
 @pytest.mark.parametrize("L,sink,local,positions", [
     (1, 64, 128, (0, 1, 3)),          # one-token prompt: no candidates
     (300, 256, 128, (299, 310)),      # sink covers the candidate range
@@ -159,6 +176,7 @@ def test_degenerate_geometry(L, sink, local, positions):
         dec.compare(_queries(1, 2, 400 + i), pos)
 
 
+@pytest.mark.gpu_pending
 def test_repeated_calls_are_identical():
     L, cap = 1200, 1300
     w = C0_TINY.with_(heads_q=4, heads_kv=2, sink=64, local=256)
@@ -173,6 +191,7 @@ def test_repeated_calls_are_identical():
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
+@pytest.mark.gpu_pending
 def test_llama_128k_layer():
     w = C2_LLAMA_128K
     L = w.seq_len
