@@ -25,7 +25,9 @@ MODES = {"anchor": SPA_MODE_ANCHOR, "sale": SPA_MODE_SALE, "dense": SPA_MODE_DEN
 
 EXPORTED = ("sparse_prefill_workspace_bytes", "sparse_prefill_plan", "sparse_prefill_attn",
             "sparse_prefill_stats", "sparse_prefill_status_string", "sparse_prefill_plan_static",
-            "sparse_decode_scratch_bytes", "sparse_decode_prepare", "sparse_decode_attn")
+            "sparse_decode_scratch_bytes", "sparse_decode_prepare", "sparse_decode_attn",
+            "sparse_fp8_scales_floats", "sparse_fp8_scratch_bytes", "sparse_fp8_quantize",
+            "sparse_prefill_attn_fp8")
 
 
 class SpaParams(ctypes.Structure):
@@ -83,6 +85,14 @@ def _load():
     lib.sparse_decode_prepare.restype = ctypes.c_int
     lib.sparse_decode_attn.argtypes = [P, vp, vp, vp, i32, i32, vp, sz, vp, sz, vp, vp, vp]
     lib.sparse_decode_attn.restype = ctypes.c_int
+    lib.sparse_fp8_scales_floats.argtypes = [P]
+    lib.sparse_fp8_scales_floats.restype = sz
+    lib.sparse_fp8_scratch_bytes.argtypes = [P]
+    lib.sparse_fp8_scratch_bytes.restype = sz
+    lib.sparse_fp8_quantize.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sparse_fp8_quantize.restype = ctypes.c_int
+    lib.sparse_prefill_attn_fp8.argtypes = [P, vp, vp, vp, vp, vp, sz, vp, vp, vp]
+    lib.sparse_prefill_attn_fp8.restype = ctypes.c_int
     lib.sparse_prefill_status_string.argtypes = [ctypes.c_int]
     lib.sparse_prefill_status_string.restype = ctypes.c_char_p
     return lib
@@ -194,6 +204,32 @@ def sparse_decode_attn(params: SpaParams, q, k_cache, v_cache, kv_capacity: int,
     return int(_lib.sparse_decode_attn(ctypes.byref(params), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                        int(kv_capacity), int(pos), _ptr(workspace), wb,
                                        _ptr(scratch), sb, _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def sparse_fp8_scales_floats(params: SpaParams) -> int:
+    return int(_lib.sparse_fp8_scales_floats(ctypes.byref(params)))
+
+
+def sparse_fp8_scratch_bytes(params: SpaParams) -> int:
+    return int(_lib.sparse_fp8_scratch_bytes(ctypes.byref(params)))
+
+
+def sparse_fp8_quantize(params: SpaParams, q, k, v, q8, k8, v8, scales, scratch,
+                        scratch_bytes=None, stream=None) -> int:
+    """E4M3 codes of q, k (mean-smoothed), v and their scales (layout in spa.h)."""
+    sb = _nbytes(scratch) if scratch_bytes is None else int(scratch_bytes)
+    return int(_lib.sparse_fp8_quantize(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(q8),
+                                        _ptr(k8), _ptr(v8), _ptr(scales), _ptr(scratch), sb,
+                                        _stream(stream)))
+
+
+def sparse_prefill_attn_fp8(params: SpaParams, q8, k8, v8, scales, workspace, o, lse=None,
+                            workspace_bytes=None, stream=None) -> int:
+    """Attention over the plan's kept keys with E4M3 operands."""
+    wb = _nbytes(workspace) if workspace_bytes is None else int(workspace_bytes)
+    return int(_lib.sparse_prefill_attn_fp8(ctypes.byref(params), _ptr(q8), _ptr(k8), _ptr(v8),
+                                            _ptr(scales), _ptr(workspace), wb, _ptr(o), _ptr(lse),
+                                            _stream(stream)))
 
 
 def sparse_prefill_status_string(status: int) -> str:

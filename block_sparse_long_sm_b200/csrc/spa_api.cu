@@ -12,6 +12,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/spa.h"
+#include "fp8_quant.cuh"
 #include "host.cuh"
 #include "ptx.cuh"
 #include "sale.cuh"
@@ -20,6 +21,28 @@
 namespace {
 
 using namespace spa;
+
+// FP8 quantisation: the scales array (documented in spa.h) and the scratch.
+struct Fp8Layout {
+  long long qs = 0, ks = 0, vs = 0, kmean = 0, floats = 0;   // float offsets
+  size_t kpart = 0, kabs = 0, vabs = 0, scratch = 0;        // byte offsets
+};
+
+Fp8Layout fp8_layout(const spa_params* p) {
+  Fp8Layout f;
+  const long long nqb = (p->seq_len + 127) / 128;
+  const long long bh = (long long)p->batch * p->heads_q, bkv = (long long)p->batch * p->heads_kv;
+  f.qs = 0;
+  f.ks = bh * nqb;
+  f.vs = f.ks + bkv;
+  f.kmean = f.vs + bkv * 128;
+  f.floats = f.kmean + bkv * 128;
+  f.kpart = 0;
+  f.kabs = align_up((size_t)bkv * kKmeanChunks * 128 * 8);
+  f.vabs = align_up(f.kabs + (size_t)bkv * 4);
+  f.scratch = align_up(f.vabs + (size_t)bkv * 128 * 4);
+  return f;
+}
 
 }  // namespace
 
@@ -327,6 +350,51 @@ SPA_API spa_status sparse_prefill_plan_static(const spa_params* p, const void* q
       cudaMemcpyAsync(error_word, err, sizeof(uint32_t), cudaMemcpyDeviceToDevice, stream) !=
           cudaSuccess)
     return SPA_ERR_CUDA;
+  return SPA_OK;
+}
+
+SPA_API size_t sparse_fp8_scales_floats(const spa_params* p) {
+  if (validate(p) != SPA_OK) return 0;
+  return (size_t)fp8_layout(p).floats;
+}
+
+SPA_API size_t sparse_fp8_scratch_bytes(const spa_params* p) {
+  if (validate(p) != SPA_OK) return 0;
+  return fp8_layout(p).scratch;
+}
+
+SPA_API spa_status sparse_fp8_quantize(const spa_params* p, const void* q, const void* k,
+                                       const void* v, void* q8, void* k8, void* v8,
+                                       float* scales, void* scratch, size_t scratch_bytes,
+                                       cudaStream_t stream) {
+  spa_status st = validate(p);
+  if (st != SPA_OK) return st;
+  const Fp8Layout f = fp8_layout(p);
+  if (!scratch || !aligned16(scratch)) return SPA_ERR_INVALID;
+  if (scratch_bytes < f.scratch) return SPA_ERR_WORKSPACE;
+  const int B = p->batch, L = p->seq_len;
+  if (B == 0 || L == 0) return SPA_OK;
+  if (!q || !k || !v || !q8 || !k8 || !v8 || !scales || !aligned16(q) || !aligned16(k) ||
+      !aligned16(v) || !aligned16(q8) || !aligned16(k8) || !aligned16(v8) || !aligned16(scales))
+    return SPA_ERR_INVALID;
+  const long long BH = (long long)B * p->heads_q, BKV = (long long)B * p->heads_kv;
+  const int nqb = (L + 127) / 128;
+  uint8_t* sc = static_cast<uint8_t*>(scratch);
+  KmeanArgs ka{static_cast<const __nv_bfloat16*>(k), L, reinterpret_cast<double*>(sc + f.kpart),
+               scales + f.kmean};
+  kmean_partial_kernel<<<dim3(kKmeanChunks, (unsigned)BKV), 128, 0, stream>>>(ka);
+  kmean_final_kernel<<<(unsigned)BKV, 128, 0, stream>>>(ka);
+  if (cudaMemsetAsync(sc + f.kabs, 0, f.scratch - f.kabs, stream) != cudaSuccess)
+    return SPA_ERR_CUDA;
+  Fp8QuantArgs a{static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                 static_cast<const __nv_bfloat16*>(v), scales + f.kmean, L, nqb,
+                 static_cast<uint8_t*>(q8), static_cast<uint8_t*>(k8), static_cast<uint8_t*>(v8),
+                 scales + f.qs, scales + f.ks, scales + f.vs,
+                 reinterpret_cast<uint32_t*>(sc + f.kabs), reinterpret_cast<uint32_t*>(sc + f.vabs)};
+  fp8_quant_q_kernel<<<dim3(nqb, (unsigned)BH), 128, 0, stream>>>(a);
+  fp8_kv_absmax_kernel<<<dim3(kFp8Chunks, (unsigned)BKV), 128, 0, stream>>>(a);
+  fp8_kv_quant_kernel<<<dim3(kFp8Chunks, (unsigned)BKV), 128, 0, stream>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   return SPA_OK;
 }
 

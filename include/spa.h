@@ -249,6 +249,44 @@ SPA_API spa_status sparse_decode_attn(const spa_params* p, const void* q, const 
                                       size_t scratch_bytes, void* o, float* lse,
                                       cudaStream_t stream);
 
+/* FP8 attention (SALE's Computation Pass on quantised operands,
+ * "SageAttention-style": the review of SALE, Summary), on the tcgen05
+ * kind::f8f6f4 tensor cores.  Two calls:
+ *
+ * sparse_fp8_quantize writes E4M3 codes (OCP "fn": bias 7, 3 mantissa bits,
+ * largest finite 448; round to nearest even, saturating) of q, k, v:
+ *   q8       uint8 [B, Hq, L, 128], one scale per (b, q head, 128-row block);
+ *   k8       uint8 [B, Hkv, L, 128] of K minus its per-(b, kv head) sequence
+ *            mean (fp64 sum / L rounded once to fp32; a constant shift of each
+ *            row's scores), one scale per (b, kv head);
+ *   v8       uint8 [B, Hkv, L, 128], one scale per (b, kv head, channel);
+ *   scales   fp32 [sparse_fp8_scales_floats(p)] = q scales [B*Hq*nqb], k scales
+ *            [B*Hkv], v scales [B*Hkv*128], K means [B*Hkv*128], in that order;
+ * scale = absmax / 448 in IEEE fp32 (1 for an all-zero group); code =
+ * E4M3(x / scale) with an IEEE fp32 division.  scratch: device buffer of
+ * sparse_fp8_scratch_bytes(p), 16-byte aligned, contents not kept.
+ *
+ * sparse_prefill_attn_fp8 runs the attention of sparse_prefill_attn over the
+ * plan in the workspace (mode, sink, local as planned) with the dequantised
+ * operands: P is rounded to E4M3 before the PV product (relative error
+ * <= 2^-4 each), O is bf16 [B, Hq, L, 128], and lse (optional, fp32
+ * [B, Hq, L], natural log) is that of the scores against the unsmoothed
+ * dequantised keys (the mean shift is added back).
+ *
+ * Pointers are device pointers, 16-byte aligned (scales and lse 4-byte).
+ * Argument errors are returned before any launch; device-side errors set the
+ * workspace error word as for sparse_prefill_attn. */
+SPA_API size_t sparse_fp8_scales_floats(const spa_params* p);
+SPA_API size_t sparse_fp8_scratch_bytes(const spa_params* p);
+SPA_API spa_status sparse_fp8_quantize(const spa_params* p, const void* q, const void* k,
+                                       const void* v, void* q8, void* k8, void* v8,
+                                       float* scales, void* scratch, size_t scratch_bytes,
+                                       cudaStream_t stream);
+SPA_API spa_status sparse_prefill_attn_fp8(const spa_params* p, const void* q8, const void* k8,
+                                           const void* v8, const float* scales, void* workspace,
+                                           size_t workspace_bytes, void* o, float* lse,
+                                           cudaStream_t stream);
+
 /* Static string for a status code. */
 SPA_API const char* sparse_prefill_status_string(spa_status s);
 

@@ -146,3 +146,29 @@ def test_decode_validation_before_any_launch():
     bad = spa.make_params(1, 4, 2, 1024, sink=64, local=100)
     assert spa.sparse_decode_prepare(bad, 1100, A, S, workspace_bytes=ws, scratch_bytes=sc,
                                      stream=0) == spa.SPA_ERR_INVALID
+
+
+def test_fp8_sizes_and_validation_before_any_launch():
+    p = spa.make_params(2, 8, 2, 1000, sink=64, local=128)
+    nqb = 8
+    assert spa.sparse_fp8_scales_floats(p) == 2 * 8 * nqb + 2 * 2 + 2 * (2 * 2 * 128)
+    sc = spa.sparse_fp8_scratch_bytes(p)
+    assert sc >= 2 * 2 * 64 * 128 * 8 + 4 * 2 * 2 * 128
+    bad = spa.make_params(2, 8, 2, 1000, sink=64, local=100)
+    assert spa.sparse_fp8_scales_floats(bad) == 0 and spa.sparse_fp8_scratch_bytes(bad) == 0
+    A = 1 << 20
+    assert spa.sparse_fp8_quantize(p, A, A, A, A, A, A, A, A, scratch_bytes=sc - 1,
+                                   stream=0) == spa.SPA_ERR_WORKSPACE
+    assert spa.sparse_fp8_quantize(p, 0, A, A, A, A, A, A, A, scratch_bytes=sc,
+                                   stream=0) == spa.SPA_ERR_INVALID
+    assert spa.sparse_fp8_quantize(p, A, A, A, A + 8, A, A, A, A, scratch_bytes=sc,
+                                   stream=0) == spa.SPA_ERR_INVALID
+    assert spa.sparse_fp8_quantize(bad, A, A, A, A, A, A, A, A, scratch_bytes=sc,
+                                   stream=0) == spa.SPA_ERR_INVALID
+    ws = spa.sparse_prefill_workspace_bytes(p)
+    assert spa.sparse_prefill_attn_fp8(p, A, A, A, A, A, A, workspace_bytes=ws - 1,
+                                       stream=0) == spa.SPA_ERR_WORKSPACE
+    assert spa.sparse_prefill_attn_fp8(p, A, A, A, A + 2, A, A, workspace_bytes=ws,
+                                       stream=0) == spa.SPA_ERR_INVALID
+    assert spa.sparse_prefill_attn_fp8(p, A, 0, A, A, A, A, workspace_bytes=ws,
+                                       stream=0) == spa.SPA_ERR_INVALID
