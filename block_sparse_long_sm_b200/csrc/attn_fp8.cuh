@@ -458,7 +458,9 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
             }
           }
         }
-        if (row < a.L && a.lse != nullptr) {
+        // the Q tile is read with generic loads: observe its TMA completion
+        if (a.lse != nullptr && !warp_wait(bar_q, 0, wc)) ok = false;
+        if (ok && row < a.L && a.lse != nullptr) {
           // q^_r . mu from row r of the swizzled Q code tile
           float dot = 0.f;
 #pragma unroll 4
