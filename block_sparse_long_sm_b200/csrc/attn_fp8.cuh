@@ -29,6 +29,7 @@
 #include "common.cuh"
 #include "fp8_cvt.cuh"
 #include "ptx.cuh"
+#include "tiles.cuh"
 
 namespace spa {
 
@@ -64,15 +65,9 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
 }
 
 struct F8Args {
-  int B, Hq, Hkv, L, nqb, group;
-  int sink, local, mode;
+  TileGeom g;                 // block geometry and the plan's lists
   float sl2;                  // softmax scale * log2(e), before the quantisation scales
   float scale;                // softmax scale (natural units), for the LSE shift
-  const int* counts;
-  const int* lists;
-  long long list_per_head;
-  long long cap_a;
-  int list_unit;
   const float* qs;            // [B*Hq][nqb]
   const float* ks;            // [B*Hkv]
   const float* vs;            // [B*Hkv][128]
@@ -82,66 +77,6 @@ struct F8Args {
   uint32_t* err;
   uint64_t wait_ns;
 };
-
-// The block's tiles in the order of the bf16 kernel: sink, selected, local.
-struct F8Item {
-  int b, h, kvh, qb, row0, le, ls, sink_end;
-  int n_sink_t, n_sel_t, n_loc_t, n_sel, loc_start;
-  long long list_off;
-};
-
-__device__ __forceinline__ F8Item f8_item(const F8Args& a, int x) {
-  F8Item it;
-  const int per_kv = a.nqb * a.group;
-  const int bkv = x / per_kv;
-  const int rem = x - bkv * per_kv;
-  it.qb = a.nqb - 1 - rem / a.group;           // longest blocks first
-  it.b = bkv / a.Hkv;
-  it.kvh = bkv - it.b * a.Hkv;
-  it.h = it.kvh * a.group + rem % a.group;
-  it.row0 = it.qb * 128;
-  it.le = min(it.row0 + 128, a.L);
-  it.ls = max(0, it.row0 + 128 - a.local);
-  it.sink_end = min(a.sink, it.ls);
-  if (a.mode == kModeDense) {
-    it.n_sink_t = 0;
-    it.n_sel = 0;
-    it.loc_start = 0;
-    it.list_off = 0;
-  } else {
-    it.n_sink_t = (it.sink_end + 127) / 128;
-    const int bh = it.b * a.Hq + it.h;
-    it.n_sel = a.counts[(long long)bh * a.nqb + it.qb] * a.list_unit;
-    it.loc_start = it.ls;
-    it.list_off = (long long)bh * a.list_per_head + cap_prefix(it.qb, 128, a.cap_a) / a.list_unit;
-  }
-  it.n_sel_t = (it.n_sel + 127) / 128;
-  it.n_loc_t = (it.le - it.loc_start + 127) / 128;
-  return it;
-}
-
-struct F8Tile {
-  int gather, key0, valid, causal;
-};
-
-__device__ __forceinline__ F8Tile f8_tile(const F8Item& it, int t) {
-  F8Tile d;
-  if (t < it.n_sink_t) {
-    d = {0, t * 128, min(128, it.sink_end - t * 128), 0};
-  } else if (t < it.n_sink_t + it.n_sel_t) {
-    const int k0 = (t - it.n_sink_t) * 128;
-    d = {1, k0, min(128, it.n_sel - k0), 0};
-  } else {
-    const int k0 = it.loc_start + (t - it.n_sink_t - it.n_sel_t) * 128;
-    d = {0, k0, min(128, it.le - k0), k0 == it.row0 ? 1 : 0};
-  }
-  return d;
-}
-
-__device__ __forceinline__ int f8_sel_key(const F8Args& a, const F8Item& it, int n) {
-  if (a.list_unit == 1) return a.lists[it.list_off + n];
-  return a.lists[it.list_off + n / a.list_unit] * a.list_unit + n % a.list_unit;
-}
 
 __global__ void __launch_bounds__(kF8Threads, 1)
 sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
@@ -205,9 +140,9 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_vg);
   }
-  const F8Item it = f8_item(a, blockIdx.x);
+  const BlockTiles it = block_tiles(a.g, blockIdx.x);
   if (threadIdx.x >= 64) {
-    const long long c = (long long)(it.b * a.Hkv + it.kvh) * 128 + threadIdx.x - 64;
+    const long long c = (long long)(it.b * a.g.Hkv + it.kvh) * 128 + threadIdx.x - 64;
     vscale[threadIdx.x - 64] = a.vs[c];
     kmu[threadIdx.x - 64] = a.kmean[c];
   }
@@ -218,23 +153,23 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
   const WaitCtx wc{abort_flag, a.err, a.wait_ns};
 
   const int T = it.n_sink_t + it.n_sel_t + it.n_loc_t;
-  const int kv_row0 = (it.b * a.Hkv + it.kvh) * a.L;
+  const int kv_row0 = (it.b * a.g.Hkv + it.kvh) * a.g.L;
 
   if (warp == 0) {
     // ------------------------------------------------------------- producer
     int issued = 0;
     if (lane == 0) {
       mbar_arrive_expect_tx(bar_q, kTile8);
-      tma_load_2d(s_q, &tm_q, bar_q, 0, (it.b * a.Hq + it.h) * a.L + it.row0);
+      tma_load_2d(s_q, &tm_q, bar_q, 0, (it.b * a.g.Hq + it.h) * a.g.L + it.row0);
     }
     auto fetch = [&](int t, int (&j)[4], int& first) {
-      const F8Tile td = f8_tile(it, t);
+      const Tile td = tile_of(it, t);
       if (!td.gather) return;
-      first = f8_sel_key(a, it, td.key0);
+      first = selected_key(a.g, it, td.key0);
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const int row = lane * 4 + r;
-        j[r] = row < td.valid ? f8_sel_key(a, it, td.key0 + row) : first;
+        j[r] = row < td.valid ? selected_key(a.g, it, td.key0 + row) : first;
       }
     };
     int nj[4] = {0, 0, 0, 0}, nfirst = 0;
@@ -247,7 +182,7 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (t >= kF8Stages) {
         if (!warp_wait(bar_empty(st), ((t / kF8Stages) - 1) & 1, wc)) break;
       }
-      const F8Tile td = f8_tile(it, t);
+      const Tile td = tile_of(it, t);
       const uint32_t kf = bar_kfull(st), vf = bar_vfull(st);
       if (!td.gather) {
         if (lane == 0) {
@@ -260,7 +195,7 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         bool bad = false;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          if (j[r] < 0 || j[r] >= a.L) {
+          if (j[r] < 0 || j[r] >= a.g.L) {
             bad = true;
             j[r] = 0;
           }
@@ -268,7 +203,7 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (bad) atomicOr(a.err, kErrBadIndex);
         const int last = __shfl_sync(0xffffffffu, j[3], 31);
         const bool contiguous = (td.valid == 128) && (last - first == 127) && first >= 0 &&
-                                first < a.L && last < a.L;
+                                first < a.g.L && last < a.g.L;
         if (lane == 0) {
           mbar_arrive_expect_tx(kf, kTile8);
           mbar_arrive_expect_tx(vf, kTile8);
@@ -340,8 +275,9 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    const int bh = it.b * a.Hq + it.h;
-    const float sl2 = a.sl2 * a.qs[(long long)bh * a.nqb + it.qb] * a.ks[it.b * a.Hkv + it.kvh];
+    const int bh = it.b * a.g.Hq + it.h;
+    const float sl2 =
+        a.sl2 * a.qs[(long long)bh * a.g.nqb + it.qb] * a.ks[it.b * a.g.Hkv + it.kvh];
     float m_used = -INFINITY;
     float lsum = 0.f;
     bool ok = true;
@@ -356,7 +292,7 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_before();
       mbar_arrive(bar_sfree0 + 8u * b);
 
-      const F8Tile td = f8_tile(it, t);
+      const Tile td = tile_of(it, t);
       const int limit = td.causal ? min(td.valid, r + 1) : td.valid;
       float mxv[8];
 #pragma unroll
@@ -434,13 +370,13 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         tc_fence_after();
         const int row = it.row0 + r;
         const float inv = 1.0f / lsum;
-        __nv_bfloat16* orow = a.o + (((long long)bh * a.L) + row) * 128;
+        __nv_bfloat16* orow = a.o + (((long long)bh * a.g.L) + row) * 128;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t ov[32];
           tmem_ld32(tmem + lane_off + 256u + 32u * c, ov);
           tmem_ld_wait();
-          if (row < a.L) {
+          if (row < a.g.L) {
             uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c);
             const float* vsc = vscale + 32 * c;
 #pragma unroll
@@ -460,7 +396,7 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         // the Q tile is read with generic loads: observe its TMA completion
         if (a.lse != nullptr && !warp_wait(bar_q, 0, wc)) ok = false;
-        if (ok && row < a.L && a.lse != nullptr) {
+        if (ok && row < a.g.L && a.lse != nullptr) {
           // q^_r . mu from row r of the swizzled Q code tile
           float dot = 0.f;
 #pragma unroll 4
@@ -478,8 +414,8 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
               dot = fmaf(hi.y, mu[3], dot);
             }
           }
-          const float q_scale = a.qs[(long long)bh * a.nqb + it.qb];
-          a.lse[(long long)bh * a.L + row] = (m_used - kF8PShift) * 0.69314718055994531f +
+          const float q_scale = a.qs[(long long)bh * a.g.nqb + it.qb];
+          a.lse[(long long)bh * a.g.L + row] = (m_used - kF8PShift) * 0.69314718055994531f +
                                              logf(lsum) + a.scale * q_scale * dot;
         }
       }

@@ -11,6 +11,7 @@
 
 #include "../../include/spa.h"
 #include "common.cuh"
+#include "tiles.cuh"
 
 namespace {
 
@@ -204,6 +205,26 @@ uint64_t wait_ns(const spa_params* p) {
 template <typename K>
 cudaError_t set_smem(K kernel, uint32_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+// The plan's geometry and lists as the tile-walking kernels read them.
+TileGeom tile_geom(const spa_params* p, const Layout& lo, uint8_t* ws) {
+  TileGeom g;
+  g.Hq = p->heads_q;
+  g.Hkv = p->heads_kv;
+  g.L = p->seq_len;
+  g.nqb = lo.nqb;
+  g.group = lo.group;
+  g.sink = p->sink;
+  g.local = p->local;
+  g.mode = p->mode == SPA_MODE_ANCHOR ? kModeAnchor
+                                      : (p->mode == SPA_MODE_SALE ? kModeSale : kModeDense);
+  g.counts = reinterpret_cast<const int*>(ws + lo.counts);
+  g.lists = reinterpret_cast<const int*>(ws + lo.lists);
+  g.list_per_head = lo.list_per_head;
+  g.cap_a = lo.cap_a;
+  g.list_unit = lo.unit;
+  return g;
 }
 
 spa_status common_checks(const spa_params* p, const void* workspace, size_t ws_bytes,

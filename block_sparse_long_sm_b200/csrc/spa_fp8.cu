@@ -38,16 +38,9 @@ SPA_API spa_status sparse_prefill_attn_fp8(const spa_params* p, const void* q8, 
   // scales: qs [B*Hq*nqb], ks [B*Hkv], vs [B*Hkv*128], K mean [B*Hkv*128]
   const long long n_qs = BH * lo.nqb;
   F8Args a;
-  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.L = L; a.nqb = lo.nqb; a.group = lo.group;
-  a.sink = p->sink; a.local = p->local;
-  a.mode = p->mode == SPA_MODE_ANCHOR ? kModeAnchor : (p->mode == SPA_MODE_SALE ? kModeSale : kModeDense);
+  a.g = tile_geom(p, lo, ws);
   a.scale = eff_scale(p);
   a.sl2 = a.scale * 1.4426950408889634f;
-  a.counts = reinterpret_cast<const int*>(ws + lo.counts);
-  a.lists = reinterpret_cast<const int*>(ws + lo.lists);
-  a.list_per_head = lo.list_per_head;
-  a.cap_a = lo.cap_a;
-  a.list_unit = lo.unit;
   a.qs = scales;
   a.ks = scales + n_qs;
   a.vs = scales + n_qs + BKV;
