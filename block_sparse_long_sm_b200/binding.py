@@ -27,7 +27,7 @@ EXPORTED = ("sparse_prefill_workspace_bytes", "sparse_prefill_plan", "sparse_pre
             "sparse_prefill_stats", "sparse_prefill_status_string", "sparse_prefill_plan_static",
             "sparse_decode_scratch_bytes", "sparse_decode_prepare", "sparse_decode_attn",
             "sparse_fp8_scales_floats", "sparse_fp8_scratch_bytes", "sparse_fp8_quantize",
-            "sparse_prefill_attn_fp8")
+            "sparse_prefill_attn_fp8", "sparse_key_mass")
 
 
 class SpaParams(ctypes.Structure):
@@ -93,6 +93,8 @@ def _load():
     lib.sparse_fp8_quantize.restype = ctypes.c_int
     lib.sparse_prefill_attn_fp8.argtypes = [P, vp, vp, vp, vp, vp, sz, vp, vp, vp]
     lib.sparse_prefill_attn_fp8.restype = ctypes.c_int
+    lib.sparse_key_mass.argtypes = [P, vp, vp, vp, i32, vp, sz, vp, vp]
+    lib.sparse_key_mass.restype = ctypes.c_int
     lib.sparse_prefill_status_string.argtypes = [ctypes.c_int]
     lib.sparse_prefill_status_string.restype = ctypes.c_char_p
     return lib
@@ -230,6 +232,14 @@ def sparse_prefill_attn_fp8(params: SpaParams, q8, k8, v8, scales, workspace, o,
     return int(_lib.sparse_prefill_attn_fp8(ctypes.byref(params), _ptr(q8), _ptr(k8), _ptr(v8),
                                             _ptr(scales), _ptr(workspace), wb, _ptr(o), _ptr(lse),
                                             _stream(stream)))
+
+
+def sparse_key_mass(params: SpaParams, q, k, lse, window: int, workspace, mass,
+                    workspace_bytes=None, stream=None) -> int:
+    """Attention mass per key from the prefill rows, from the prefill LSE."""
+    wb = _nbytes(workspace) if workspace_bytes is None else int(workspace_bytes)
+    return int(_lib.sparse_key_mass(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(lse), int(window),
+                                    _ptr(workspace), wb, _ptr(mass), _stream(stream)))
 
 
 def sparse_prefill_status_string(status: int) -> str:

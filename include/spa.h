@@ -287,6 +287,25 @@ SPA_API spa_status sparse_prefill_attn_fp8(const spa_params* p, const void* q8, 
                                            size_t workspace_bytes, void* o, float* lse,
                                            cudaStream_t stream);
 
+/* Attention mass per key from the prefill rows, reusing the prefill LSE
+ * (KVpop, Sec. 3: the future attention mass of a token, from a transposed
+ * attention pass over the sparse kept sets with the sparse LSE normalisers,
+ * aggregated over the query heads that share a kv head):
+ *
+ *   mass[b, g, j] = sum over q heads h of kv head g, and over rows i whose
+ *                   kept set (as planned in the workspace) holds j and with
+ *                   i - j >= window, of exp(s_ij - lse[b, h, i]),
+ *
+ * s_ij the scaled score of q_i and k_j.  q, k as for sparse_prefill_plan;
+ * lse fp32 [B, Hq, L] (natural log; normally sparse_prefill_attn's output
+ * for the same plan); mass fp32 [B, Hkv, L], overwritten.  window >= 0, and
+ * window <= local - block_q outside DENSE mode (every selected key then lies
+ * at least that far behind every row of its block).  Errors as for
+ * sparse_prefill_attn. */
+SPA_API spa_status sparse_key_mass(const spa_params* p, const void* q, const void* k,
+                                   const float* lse, int32_t window, void* workspace,
+                                   size_t workspace_bytes, float* mass, cudaStream_t stream);
+
 /* Static string for a status code. */
 SPA_API const char* sparse_prefill_status_string(spa_status s);
 

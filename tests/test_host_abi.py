@@ -172,3 +172,18 @@ def test_fp8_sizes_and_validation_before_any_launch():
                                        stream=0) == spa.SPA_ERR_INVALID
     assert spa.sparse_prefill_attn_fp8(p, A, 0, A, A, A, A, workspace_bytes=ws,
                                        stream=0) == spa.SPA_ERR_INVALID
+
+
+def test_key_mass_validation_before_any_launch():
+    p = spa.make_params(1, 4, 2, 1000, sink=64, local=256)
+    ws = spa.sparse_prefill_workspace_bytes(p)
+    A = 1 << 20
+
+    def call(window, q=A, ws_bytes=ws, params=p):
+        return spa.sparse_key_mass(params, q, A, A, window, A, A, workspace_bytes=ws_bytes,
+                                   stream=0)
+    assert call(-1) == spa.SPA_ERR_INVALID
+    assert call(129) == spa.SPA_ERR_UNSUPPORTED             # beyond local - block_q
+    assert call(0, ws_bytes=ws - 1) == spa.SPA_ERR_WORKSPACE
+    assert call(0, q=0) == spa.SPA_ERR_INVALID
+    assert call(0, q=A + 8) == spa.SPA_ERR_INVALID
