@@ -19,8 +19,9 @@ layer (independent problems, weak scaling, no collective on the data path);
 the timed region is bracketed by barriers and the max over ranks is reported.
 
 ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only).
-``--sweep`` runs the density sweep and ``--decode`` the decode steps that
-reuse a plan; each prints its own JSON lines instead of the headline step.
+``--sweep`` runs the density sweep, ``--decode`` the decode steps that reuse
+a plan, ``--fp8`` the E4M3 attention and ``--key-mass`` the key mass from the
+prefill LSE; each prints its own JSON lines instead of the headline step.
 """
 
 from __future__ import annotations
@@ -230,6 +231,11 @@ def main():
     ap.add_argument("--decode", action="store_true",
                     help="decode-shaped reuse of the plan instead of the headline step: one "
                          "decoding query per q head per step at positions L-1, L, ...")
+    ap.add_argument("--fp8", action="store_true",
+                    help="E4M3 quantisation + FP8 attention over the plan instead of the "
+                         "headline step")
+    ap.add_argument("--key-mass", action="store_true",
+                    help="key mass from the prefill LSE over the plan instead of the headline step")
     args = ap.parse_args()
     w = CONFIGS[args.config]
     if args.sweep:
@@ -237,6 +243,9 @@ def main():
         return
     if args.decode:
         decode_bench(args, w)
+        return
+    if args.fp8 or args.key_mass:
+        variant_bench(args, w)
         return
     if args.impl == "reference":
         run_reference(args, w)
@@ -521,6 +530,96 @@ def decode_bench(args, w: Workload):
                      "peak_source": f"{peaks['src']} HBM copy bandwidth"},
         "clocks": clk.summary(),
         "gpu_launches": 2 * args.steps,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def variant_bench(args, w: Workload):
+    """FP8 attention (--fp8) or the key mass from the prefill LSE (--key-mass)
+    over the same plan as the headline step (anchor, theta, 128K layer).  The
+    plan (and, for the key mass, the bf16 attention that yields the LSE) runs
+    once, untimed; each timed step is sparse_fp8_quantize +
+    sparse_prefill_attn_fp8, or sparse_key_mass.  Inputs are larger than L2.
+    Roofline of the dominant kernel: FP8 attention on kept FLOPs (4 d per kept
+    pair) against the measured bf16 peak times 2 (the nominal fp8:bf16 ratio);
+    the key mass on 2 d per kept pair (its QK^T) against the bf16 peak."""
+    import torch
+    import block_sparse_long_sm_b200 as spa
+    world, rank, local = _dist()
+    if rank != 0:
+        return
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+    inp = generate(w)
+    to = lambda u: torch.from_numpy(np.ascontiguousarray(u).view(np.int16)).to(dev).view(torch.bfloat16)
+    q, k, v = to(inp.q), to(inp.k), to(inp.v)
+    del inp
+    B, Hq, Hkv, L = w.batch, w.heads_q, w.heads_kv, w.seq_len
+    p = spa.make_params(B, Hq, Hkv, L, mode=args.mode, sink=w.sink, local=w.local,
+                        theta=args.theta, tau=w.tau,
+                        block_k=w.block_k if args.mode == "sale" else None)
+    ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
+    spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream), "plan")
+    st, stats = spa.sparse_prefill_stats(p, ws, stream=stream)
+    spa.check(st, "stats")
+    o = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
+    peaks = _peaks()
+    if args.fp8:
+        q8 = torch.empty((B, Hq, L, 128), dtype=torch.uint8, device=dev)
+        k8 = torch.empty((B, Hkv, L, 128), dtype=torch.uint8, device=dev)
+        v8 = torch.empty((B, Hkv, L, 128), dtype=torch.uint8, device=dev)
+        scales = torch.empty(spa.sparse_fp8_scales_floats(p), dtype=torch.float32, device=dev)
+        scratch = torch.empty(spa.sparse_fp8_scratch_bytes(p), dtype=torch.uint8, device=dev)
+        quant = lambda: spa.check(spa.sparse_fp8_quantize(p, q, k, v, q8, k8, v8, scales, scratch,
+                                                          stream=stream), "fp8 quantize")
+        attn = lambda: spa.check(spa.sparse_prefill_attn_fp8(p, q8, k8, v8, scales, ws, o, None,
+                                                              stream=stream), "fp8 attn")
+        flops = spa.kept_flops(stats)
+        peak, kernel, n_launch = 2.0 * peaks["bf16_sus"], "sparse_attn_fp8_kernel", 6
+        metric = "FP8 sparse prefill attn (quantise + attn) kept-FLOP TFLOP/s"
+    else:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+        spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, lse, stream=stream), "attn")
+        mass = torch.empty((B, Hkv, L), dtype=torch.float32, device=dev)
+        quant = None
+        attn = lambda: spa.check(spa.sparse_key_mass(p, q, k, lse, 0, ws, mass, stream=stream),
+                                 "key mass")
+        flops = 2 * 128 * int(stats.kept_pairs)
+        peak, kernel, n_launch = peaks["bf16_sus"], "key_mass_kernel", 1
+        metric = "key mass from the prefill LSE, QK^T TFLOP/s on kept pairs"
+    warm = max(3, args.warmup)
+    for _ in range(warm):
+        if quant:
+            quant()
+        attn()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            if quant:
+                quant()
+            ev[i][1].record(stream)
+            attn()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize()
+    step_ms = statistics.median(a.elapsed_time(c) for a, _, c in ev)
+    kern_ms = statistics.median(b.elapsed_time(c) for _, b, c in ev)
+    achieved = flops / (kern_ms / 1e3) / 1e12
+    line = {
+        "metric": metric, "value": flops / (step_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": warm, "ms_per_step": step_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if args.fp8 else "bf16", "data": "synthetic",
+        "config": _config(w, args), "kernel_ms": kern_ms,
+        "kept_fraction": stats.kept_pairs / stats.dense_pairs,
+        "roofline": {"bound": "tensor", "kernel": kernel, "achieved": achieved, "peak": peak,
+                     "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peaks['src']} bf16 dense, sustained"
+                                    + (" x 2 (nominal fp8:bf16)" if args.fp8 else "")},
+        "clocks": clk.summary(),
+        "gpu_launches": n_launch * args.steps,
     }
     print(json.dumps(line), flush=True)
 
