@@ -206,7 +206,8 @@ def run_reference(args, w: Workload):
 
 
 def _config(w: Workload, args):
-    return {"workload": w.name, "batch": w.batch, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
+    return {"workload": w.name, "attn_variant": "window_tiles" if getattr(args, "window_tiles", False)
+            else "gather_tiles", "batch": w.batch, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
             "seq_len": w.seq_len, "head_dim": 128, "causal": True, "mode": args.mode,
             "theta": args.theta, "sink": w.sink, "local": w.local, "block_q": 128,
             "l2": f"inputs ({2 * 128 * w.seq_len * w.batch * (w.heads_q + 2 * w.heads_kv) / 1e9:.2f} GB) "
@@ -234,6 +235,9 @@ def main():
     ap.add_argument("--fp8", action="store_true",
                     help="E4M3 quantisation + FP8 attention over the plan instead of the "
                          "headline step")
+    ap.add_argument("--window-tiles", action="store_true",
+                    help="paired attention with contiguous masked windows for near-dense "
+                         "selected keys (SPA_DEBUG_WINDOW_TILES)")
     ap.add_argument("--key-mass", action="store_true",
                     help="key mass from the prefill LSE over the plan instead of the headline step")
     args = ap.parse_args()
@@ -275,7 +279,8 @@ def main():
     B, Hq, Hkv, L = w.batch, w.heads_q, w.heads_kv, w.seq_len
     o = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
     p = spa.make_params(B, Hq, Hkv, L, mode=args.mode, sink=w.sink, local=w.local,
-                        theta=args.theta, tau=w.tau, block_k=w.block_k if args.mode == "sale" else None)
+                        theta=args.theta, tau=w.tau, block_k=w.block_k if args.mode == "sale" else None,
+                        debug_flags=spa.SPA_DEBUG_WINDOW_TILES if args.window_tiles else 0)
     ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
 
     def step():

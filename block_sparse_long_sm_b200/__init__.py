@@ -11,12 +11,13 @@ ImportError (there is no fallback).
 import importlib
 
 _BINDING_NAMES = (
-    "EXPORTED", "LIB_PATH", "MODES", "SPA_DEBUG_STALL_ATTN", "SPA_ERR_CUDA", "SPA_ERR_INVALID",
-    "SPA_ERR_TIMEOUT", "SPA_ERR_UNSUPPORTED", "SPA_ERR_WORKSPACE", "SPA_MODE_ANCHOR",
-    "SPA_MODE_DENSE", "SPA_MODE_SALE", "SPA_OK", "SpaError", "SpaParams", "SpaStats", "check",
-    "kept_flops", "make_params", "sparse_decode_attn", "sparse_decode_prepare",
-    "sparse_decode_scratch_bytes", "sparse_fp8_quantize", "sparse_fp8_scales_floats",
-    "sparse_fp8_scratch_bytes", "sparse_key_mass", "sparse_prefill_attn", "sparse_prefill_attn_fp8", "sparse_prefill_plan",
+    "EXPORTED", "LIB_PATH", "MODES", "SPA_DEBUG_STALL_ATTN", "SPA_DEBUG_WINDOW_TILES",
+    "SPA_ERR_CUDA", "SPA_ERR_INVALID", "SPA_ERR_TIMEOUT", "SPA_ERR_UNSUPPORTED",
+    "SPA_ERR_WORKSPACE", "SPA_MODE_ANCHOR", "SPA_MODE_DENSE", "SPA_MODE_SALE", "SPA_OK",
+    "SpaError", "SpaParams", "SpaStats", "check", "kept_flops", "make_params",
+    "sparse_decode_attn", "sparse_decode_prepare", "sparse_decode_scratch_bytes",
+    "sparse_fp8_quantize", "sparse_fp8_scales_floats", "sparse_fp8_scratch_bytes",
+    "sparse_key_mass", "sparse_prefill_attn", "sparse_prefill_attn_fp8", "sparse_prefill_plan",
     "sparse_prefill_plan_static", "sparse_prefill_stats", "sparse_prefill_status_string",
     "sparse_prefill_workspace_bytes")
 

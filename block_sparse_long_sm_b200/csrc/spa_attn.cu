@@ -6,6 +6,7 @@
 #include "../../include/spa.h"
 #include "attn.cuh"
 #include "attn_pair.cuh"
+#include "attn_pair_win.cuh"
 #include "host.cuh"
 
 namespace {
@@ -54,7 +55,11 @@ SPA_API spa_status sparse_prefill_attn(const spa_params* p, const void* q, const
   aa.err = reinterpret_cast<uint32_t*>(ws);
   aa.wait_ns = wait_ns(p);
   aa.debug = p->debug_flags;
-  if (lo.paired) {
+  if (lo.paired && (p->debug_flags & SPA_DEBUG_WINDOW_TILES)) {
+    if (set_smem(sparse_attn_pair_win_kernel, kPairSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
+    sparse_attn_pair_win_kernel<<<(unsigned)(lo.nb / 2), kPairThreads, kPairSmemBytes, stream>>>(
+        tq, tk, tkg, tv, tvg, aa);
+  } else if (lo.paired) {
     if (set_smem(sparse_attn_pair_kernel, kPairSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
     sparse_attn_pair_kernel<<<(unsigned)(lo.nb / 2), kPairThreads, kPairSmemBytes, stream>>>(
         tq, tk, tkg, tv, tvg, aa);

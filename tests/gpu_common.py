@@ -38,13 +38,14 @@ class Run:
 
     def __init__(self, inputs: Inputs, *, mode: str, sink: int, local: int, theta: float = 5.0,
                  tau: float = 1e-3, block_k=None, do_attn: bool = True, lse: bool = True,
-                 dev=None, step: int = 1):
+                 dev=None, step: int = 1, debug_flags: int = 0):
         B, Hq, L, _ = inputs.q.shape
         Hkv = inputs.k.shape[1]
         self.B, self.Hq, self.Hkv, self.L = B, Hq, Hkv, L
         self.group = Hq // Hkv
         self.params = spa.make_params(B, Hq, Hkv, L, mode=mode, sink=sink, local=local,
-                                      theta=theta, tau=tau, block_k=block_k, step=step)
+                                      theta=theta, tau=tau, block_k=block_k, step=step,
+                                      debug_flags=debug_flags)
         self.q, self.k, self.v = dev if dev is not None else (
             to_dev(inputs.q), to_dev(inputs.k), to_dev(inputs.v))
         nbytes = spa.sparse_prefill_workspace_bytes(self.params)
