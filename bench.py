@@ -243,7 +243,7 @@ def main():
     args = ap.parse_args()
     w = CONFIGS[args.config]
     if args.sweep:
-        sweep()
+        sweep(window_tiles=args.window_tiles)
         return
     if args.decode:
         decode_bench(args, w)
@@ -360,7 +360,7 @@ def main():
         dist.destroy_process_group()
 
 
-def sweep():
+def sweep(window_tiles: bool = False):
     """Kept fraction vs time and vs tensor peak over theta (the density sweep
     of the 128K Llama layer, its B = 4, L = 16384 variant and the 64K Qwen
     layer with half its kv heads diffuse).  One JSON line per point; theta =
@@ -406,7 +406,8 @@ def sweep():
         del wsd
         for theta in thetas:
             p = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=w.sink, local=w.local,
-                                theta=theta)
+                                theta=theta,
+                                debug_flags=spa.SPA_DEBUG_WINDOW_TILES if window_tiles else 0)
             ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
             plan_ms = timed(lambda: spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream)))
             attn_ms = timed(lambda: spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None,
@@ -417,6 +418,7 @@ def sweep():
             alg_bytes = 2 * B * Hq * L * 128 + 2 * B * Hkv * L * 128 + 4 * s.kept_candidates
             print(json.dumps({
                 "sweep": "density", "workload": w.name, "theta": theta,
+                "attn_variant": "window_tiles" if window_tiles else "gather_tiles",
                 "kept_fraction": s.kept_pairs / s.dense_pairs,
                 "kept_candidates_fraction": s.kept_candidates / max(1, s.candidates),
                 "plan_ms": plan_ms, "attn_ms": attn_ms, "step_ms": plan_ms + attn_ms,
