@@ -107,16 +107,19 @@ def _check_outputs(fr: Fp8Run, inp, b, h, rows):
     assert lse_err <= LSE_ABS, lse_err
 
 
-@pytest.mark.parametrize("mode,L,theta,bk", [("anchor", 1000, 2.5, None), ("anchor", 129, 3.0, None),
-                                             ("sale", 1500, 0.0, 32), ("dense", 700, 0.0, None)])
-def test_fp8_quantisation_and_attention(mode, L, theta, bk):
-    w = C0_TINY.with_(heads_q=4, heads_kv=2, sink=64, local=256)
+# Hq / Hkv = 2: the paired schedule (two q heads per CTA over the union
+# lists); 3: the one-head schedule (also every DENSE call).
+@pytest.mark.parametrize("mode,L,theta,bk,hq", [
+    ("anchor", 1000, 2.5, None, 4), ("anchor", 129, 3.0, None, 4), ("sale", 1500, 0.0, 32, 4),
+    ("dense", 700, 0.0, None, 4), ("anchor", 1000, 2.5, None, 6), ("sale", 900, 0.0, 64, 6)])
+def test_fp8_quantisation_and_attention(mode, L, theta, bk, hq):
+    w = C0_TINY.with_(heads_q=hq, heads_kv=2, sink=64, local=256)
     inp = generate(w, seq_len=L)
     run = Run(inp, mode=mode, sink=64, local=256, theta=theta, tau=1e-2, block_k=bk,
               do_attn=False)
     fr = Fp8Run(run)
-    for h in range(4):
+    for h in range(hq):
         _check_quantisation(fr, inp, 0, h)
     rows = sorted(set(range(0, L, max(1, L // 40))) | {L - 1, min(L - 1, 127), min(L - 1, 128)})
-    for h in (0, 3):
+    for h in (0, 1, hq - 1):
         _check_outputs(fr, inp, 0, h, rows)
