@@ -14,10 +14,12 @@
 // Attention over a key set does not depend on the order of its tiles, so the
 // result is the paired kernel's up to rounding.
 //
-// The number of selected tiles now depends on the keys, so the producer
-// counts them with one pass over the union list before the pipeline starts.
-// Everything else (roles, barriers, TMEM layout, softmax) is the paired
-// kernel's.
+// The number of selected tiles now depends on the keys.  Rather than count
+// them up front (a chain of dependent list reads), the producer publishes for
+// every tile, through the tag barrier of its V slot, a descriptor (valid
+// columns, causal, masked, last) beside the head masks; the MMA warp and the
+// softmax warps stop after the tile marked last.  Everything else (roles,
+// barriers, TMEM layout, softmax) is the paired kernel's.
 #pragma once
 
 #include "attn_pair.cuh"
@@ -132,43 +134,16 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
     window = cnt >= kWinMin;
     return window ? cnt : min(128, n_total - n);
   };
-  int* n_sel_slot = reinterpret_cast<int*>(bar_area + 520);
-  if (warp == 8) {
-    int nt = 0;
-    for (int n = 0; n < n_total; ++nt) {
-      int j[4];
-      uint32_t tg[4];
-      fetch_at(n, j, tg);
-      bool window;
-      int k0;
-      n += decide(n, j, window, k0);
-    }
-    if (lane == 0) *n_sel_slot = nt;
-  }
-  __syncthreads();
-  const int n_sel_t = *n_sel_slot;
-  const int T = it.n_sink_t + n_sel_t + it.n_loc_t;
-  // Tile t: sink tiles, selected tiles (masked through the published head
-  // masks), local tiles (the last one the causal diagonal).
-  auto wdesc = [&](int t) {
-    TileDesc d;
-    if (t < it.n_sink_t) {
-      d.gather = 0;
-      d.key0 = t * 128;
-      d.valid = min(128, it.sink_end - d.key0);
-      d.causal = 0;
-    } else if (t < it.n_sink_t + n_sel_t) {
-      d.gather = 1;
-      d.key0 = 0;
-      d.valid = 128;
-      d.causal = 0;
-    } else {
-      d.gather = 0;
-      d.key0 = it.loc_start + (t - it.n_sink_t - n_sel_t) * 128;
-      d.valid = min(128, it.le - d.key0);
-      d.causal = (d.key0 == it.row0);
-    }
-    return d;
+  // Per V slot, the descriptor of the tile in it: valid columns (bits 0-8),
+  // causal diagonal (9), masked through the head masks (10), last tile (11).
+  // Written by the producer before it arrives on the slot's tag barrier.
+  uint32_t* tdesc = reinterpret_cast<uint32_t*>(bar_area + 528);
+  auto unpack = [](uint32_t d, TileDesc& td, bool& last) {
+    td.valid = static_cast<int>(d & 0x1FFu);
+    td.causal = (d >> 9) & 1u;
+    td.gather = (d >> 10) & 1u;
+    td.key0 = 0;
+    last = (d >> 11) & 1u;
   };
 
   // Register split: the load/MMA warpgroup needs few registers, the softmax
@@ -194,8 +169,9 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
     int nj[4] = {0, 0, 0, 0};
     uint32_t ntg[4] = {0u, 0u, 0u, 0u};
     int n_cur = 0;                             // union ordinal of the next selected tile
-    if (n_sel_t > 0) fetch_at(0, nj, ntg);
-    for (int t = 0; t < T; ++t) {
+    int loc = 0;                               // local tiles issued
+    if (n_total > 0) fetch_at(0, nj, ntg);
+    for (int t = 0;; ++t) {
       const int ks = t % kPairKStages, vs = t % kPairVStages;
       if (t >= kPairKStages &&
           !warp_wait(bar_kempty(ks), ((t / kPairKStages) - 1) & 1, wc))
@@ -203,7 +179,27 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (t >= kPairVStages &&
           !warp_wait(bar_vempty(vs), ((t / kPairVStages) - 1) & 1, wc))
         break;
-      const TileDesc td = wdesc(t);
+      // tile t: sink tiles, then selected tiles while union keys remain, then
+      // local tiles (there is always one: the diagonal)
+      TileDesc td;
+      bool last = false;
+      if (t < it.n_sink_t) {
+        td.gather = 0;
+        td.key0 = t * 128;
+        td.valid = min(128, it.sink_end - td.key0);
+        td.causal = 0;
+      } else if (n_cur < n_total) {
+        td.gather = 1;
+        td.key0 = 0;
+        td.valid = 128;
+        td.causal = 0;
+      } else {
+        td.gather = 0;
+        td.key0 = it.loc_start + loc * 128;
+        td.valid = min(128, it.le - td.key0);
+        td.causal = (td.key0 == it.row0);
+        last = ++loc == it.n_loc_t;
+      }
       const uint32_t kf = bar_kfull(ks), vf = bar_vfull(vs);
       bool contiguous = !td.gather;
       int key0 = td.key0;
@@ -214,7 +210,7 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
         int k0;
         const int used = decide(n_cur, j, window, k0);
         n_cur += used;
-        if (t + 1 < it.n_sink_t + n_sel_t) fetch_at(n_cur, nj, ntg);   // next tile's keys
+        if (n_cur < n_total) fetch_at(n_cur, nj, ntg);   // the next selected tile's keys
         bool bad = false;
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
@@ -259,11 +255,16 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
             tags[(vs * 2 + 1) * 4 + x] = wb[x];
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_tag0 + 8u * vs);   // publishes this tile's masks
         contiguous = window;
         key0 = k0;
       }
+      // every tile publishes its descriptor (and a selected tile its masks)
+      if (lane == 0) {
+        tdesc[vs] = static_cast<uint32_t>(td.valid) | (static_cast<uint32_t>(td.causal) << 9) |
+                    (static_cast<uint32_t>(td.gather) << 10) | (last ? 1u << 11 : 0u);
+        mbar_arrive(bar_tag0 + 8u * vs);
+      }
+      __syncwarp();
       if (lane == 0) {
         mbar_arrive_expect_tx(kf, kTileBytes);
         mbar_arrive_expect_tx(vf, kTileBytes);
@@ -288,6 +289,7 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
                     kv_row0 + j[1], kv_row0 + j[2], kv_row0 + j[3]);
       }
       issued = t + 1;
+      if (last) break;
     }
     if (lane == 0) {   // no copy may still be in flight when the CTA exits
       mbar_drain(bar_q, 0, a.wait_ns);
@@ -321,7 +323,7 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
                       (t > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      if (ok && T > 0) {
+      if (ok) {
         if ((ok = mbar_wait(bar_kfull(0), 0, wc))) {
           tc_fence_after();
           qk(0, 0);
@@ -329,9 +331,14 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit(bar_kempty(0));
         }
       }
-      for (int t = 0; ok && t < T; ++t) {
+      for (int t = 0; ok; ++t) {
         const int vs = t % kPairVStages;
-        const bool more = t + 1 < T;
+        // tile t's descriptor was written before its K copy was armed, and
+        // kfull of tile t has been observed (QK(t) is issued)
+        TileDesc td_unused;
+        bool last;
+        unpack(tdesc[vs], td_unused, last);
+        const bool more = !last;
         // head A: PV(t), then QK(t+1)
         if (!(ok = mbar_wait(bar_pfull0, t & 1, wc))) break;
         if (!(ok = mbar_wait(bar_vfull(vs), (t / kPairVStages) & 1, wc))) break;
@@ -353,6 +360,7 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit(bar_kempty((t + 1) % kPairKStages));
         } else {
           mma_commit(bar_odone);
+          break;
         }
       }
       mma_commit(bar_drain);
@@ -371,19 +379,19 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float sl2 = a.sl2;
     float m_used = -INFINITY;
     float lsum = 0.f;
-    uint32_t tag_phase = 0u;                   // bit vs: phase of tag barrier vs
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
+    bool last = false;
+    for (int t = 0; !last; ++t) {
       if (!(ok = warp_wait(bar_sfull0 + 8u * hd, t & 1, wc))) break;
       tc_fence_after();
-      const TileDesc td = wdesc(t);
+      // every tile arrives once on its V slot's tag barrier
+      const int vs = t % kPairVStages;
+      if (!(ok = warp_wait(bar_tag0 + 8u * vs, (t / kPairVStages) & 1, wc))) break;
+      TileDesc td;
+      unpack(tdesc[vs], td, last);
       const int limit = td.causal ? min(td.valid, r + 1) : td.valid;
       uint32_t tw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
       if (td.gather) {
-        const int vs = t % kPairVStages;
-        // tag barrier phases of this slot count the gathered tiles that used it
-        if (!(ok = warp_wait(bar_tag0 + 8u * vs, (tag_phase >> vs) & 1u, wc))) break;
-        tag_phase ^= 1u << vs;
 #pragma unroll
         for (int w = 0; w < 4; ++w) tw[w] = tags[(vs * 2 + hd) * 4 + w];
       }
@@ -465,7 +473,7 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_before();
       mbar_arrive(bar_pfull0 + 8u * hd);
     }
-    if (ok && T > 0) {
+    if (ok) {
       ok = warp_wait(bar_odone, 0, wc);
       if (ok) {
         tc_fence_after();
