@@ -138,13 +138,6 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
   // causal diagonal (9), masked through the head masks (10), last tile (11).
   // Written by the producer before it arrives on the slot's tag barrier.
   uint32_t* tdesc = reinterpret_cast<uint32_t*>(bar_area + 528);
-  auto unpack = [](uint32_t d, TileDesc& td, bool& last) {
-    td.valid = static_cast<int>(d & 0x1FFu);
-    td.causal = (d >> 9) & 1u;
-    td.gather = (d >> 10) & 1u;
-    td.key0 = 0;
-    last = (d >> 11) & 1u;
-  };
 
   // Register split: the load/MMA warpgroup needs few registers, the softmax
   // warpgroups hold a full 128-column S row each.  Launched with 168 per
@@ -226,35 +219,18 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (bad) atomicOr(a.err, kErrBadIndex);
         // membership masks, bit c of word w <=> column 32w + c belongs to the head:
         // a window tile's column is key - k0, a gathered tile's its row 4 lane + r
-        uint32_t wa[4] = {0u, 0u, 0u, 0u}, wb[4] = {0u, 0u, 0u, 0u};
+        // (the slot's masks are free: the PV that read them has completed)
+        if (lane < 8) tags[vs * 8 + lane] = 0u;
+        __syncwarp();
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           const int ord = lane * 4 + r;
           const int col = window ? j[r] - k0 : ord;
           const bool in = window ? (ord < used) : true;   // padding rows carry tag 0
-          const uint32_t ta = in ? (tg[r] & 1u) : 0u, tb = in ? ((tg[r] >> 1) & 1u) : 0u;
-          const int w = (col >> 5) & 3, bit = col & 31;
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            wa[x] |= (x == w) ? (ta << bit) : 0u;
-            wb[x] |= (x == w) ? (tb << bit) : 0u;
-          }
+          if (in && (tg[r] & 1u)) atomicOr(&tags[(vs * 2 + 0) * 4 + (col >> 5)], 1u << (col & 31));
+          if (in && (tg[r] & 2u)) atomicOr(&tags[(vs * 2 + 1) * 4 + (col >> 5)], 1u << (col & 31));
         }
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) {
-            wa[x] |= __shfl_xor_sync(0xffffffffu, wa[x], o);
-            wb[x] |= __shfl_xor_sync(0xffffffffu, wb[x], o);
-          }
-        }
-        if (lane == 0) {
-#pragma unroll
-          for (int x = 0; x < 4; ++x) {
-            tags[(vs * 2 + 0) * 4 + x] = wa[x];
-            tags[(vs * 2 + 1) * 4 + x] = wb[x];
-          }
-        }
+        __syncwarp();
         contiguous = window;
         key0 = k0;
       }
@@ -335,10 +311,7 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int vs = t % kPairVStages;
         // tile t's descriptor was written before its K copy was armed, and
         // kfull of tile t has been observed (QK(t) is issued)
-        TileDesc td_unused;
-        bool last;
-        unpack(tdesc[vs], td_unused, last);
-        const bool more = !last;
+        const bool more = ((tdesc[vs] >> 11) & 1u) == 0u;
         // head A: PV(t), then QK(t+1)
         if (!(ok = mbar_wait(bar_pfull0, t & 1, wc))) break;
         if (!(ok = mbar_wait(bar_vfull(vs), (t / kPairVStages) & 1, wc))) break;
@@ -387,11 +360,12 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
       // every tile arrives once on its V slot's tag barrier
       const int vs = t % kPairVStages;
       if (!(ok = warp_wait(bar_tag0 + 8u * vs, (t / kPairVStages) & 1, wc))) break;
-      TileDesc td;
-      unpack(tdesc[vs], td, last);
-      const int limit = td.causal ? min(td.valid, r + 1) : td.valid;
+      const uint32_t dw = tdesc[vs];
+      last = ((dw >> 11) & 1u) != 0u;
+      const int valid = static_cast<int>(dw & 0x1FFu);
+      const int limit = ((dw >> 9) & 1u) ? min(valid, r + 1) : valid;
       uint32_t tw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      if (td.gather) {
+      if ((dw >> 10) & 1u) {
 #pragma unroll
         for (int w = 0; w < 4; ++w) tw[w] = tags[(vs * 2 + hd) * 4 + w];
       }
