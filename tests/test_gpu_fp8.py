@@ -123,3 +123,15 @@ def test_fp8_quantisation_and_attention(mode, L, theta, bk, hq):
     rows = sorted(set(range(0, L, max(1, L // 40))) | {L - 1, min(L - 1, 127), min(L - 1, 128)})
     for h in (0, 1, hq - 1):
         _check_outputs(fr, inp, 0, h, rows)
+
+
+def test_fp8_llama_32k_sampled():
+    from workloads import C1_LLAMA_32K
+    from gpu_common import sample_rows
+    w = C1_LLAMA_32K
+    inp = generate(w)
+    run = Run(inp, mode="anchor", sink=w.sink, local=w.local, theta=w.theta, do_attn=False)
+    fr = Fp8Run(run)
+    for h in (0, 13, 31):
+        _check_quantisation(fr, inp, 0, h)
+        _check_outputs(fr, inp, 0, h, sample_rows(w.seq_len, 16, h, must=(0, 128, w.seq_len - 1)))

@@ -87,3 +87,18 @@ def test_key_mass_with_the_attention_lse():
     got = _gpu_mass(run, run.lse, 0)
     rel = REL + math.expm1(2e-3)
     assert np.all(np.abs(got - ref) <= rel * ref + 1e-6)
+
+
+def test_key_mass_llama_32k_conserves_the_rows():
+    # every row's probabilities over its kept set sum to one, so the masses of
+    # a kv head sum to (its q heads) x L, up to the bf16 probabilities and the
+    # attention's LSE (both within the relative bound used above)
+    from workloads import C1_LLAMA_32K
+    w = C1_LLAMA_32K
+    inp = generate(w)
+    run = Run(inp, mode="anchor", sink=w.sink, local=w.local, theta=w.theta)
+    got = _gpu_mass(run, run.lse, 0)
+    per_kv = got.sum(axis=2)[0]
+    want = run.group * w.seq_len
+    assert np.all(np.abs(per_kv - want) <= (REL + math.expm1(2e-3)) * want), per_kv
+    assert np.all(got >= 0)
