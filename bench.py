@@ -537,8 +537,86 @@ def decode_bench(args, w: Workload):
                      "peak_source": f"{peaks['src']} HBM copy bandwidth"},
         "clocks": clk.summary(),
         "gpu_launches": 2 * args.steps,
+        "cpu_baseline": oracle_decode_sample(w, args.theta),
     }
     print(json.dumps(line), flush=True)
+
+
+def _oracle_cores():
+    cores = len(os.sched_getaffinity(0))
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        cores = max((i.get("num_threads", 1) for i in info), default=cores)
+    except Exception:
+        pass
+    return cores
+
+
+def oracle_decode_sample(w: Workload, theta: float, heads: int = 4):
+    """fp64 oracle of one decode step for the first `heads` q heads of kv head
+    0 at pos = L - 1 (their last-block anchor selection, then attention over
+    the decode key set), scaled to all q heads: decoded tokens/s."""
+    from oracle import decode as odec
+    from oracle import selection as osel
+    from workloads import bf16_bits_to_f32
+    inp = generate(w, kv_groups=[0])
+    L = w.seq_len
+    kh = bf16_bits_to_f32(inp.k[0, 0]).astype(np.float64)
+    vh = bf16_bits_to_f32(inp.v[0, 0]).astype(np.float64)
+    qb = (L - 1) // 128
+    t0 = time.perf_counter()
+    for h in range(heads):
+        qh = bf16_bits_to_f32(inp.q[0, h]).astype(np.float64)
+        sel = osel.anchor_block(qh, kh, qb, bq=128, sink=w.sink, local=w.local, theta=theta).kept
+        keys = odec.decode_keys(L - 1, L, sel, bq=128, sink=w.sink, local=w.local)
+        odec.decode_attend(qh[L - 1], kh, vh, keys)
+    dt = time.perf_counter() - t0
+    per_step = dt * w.heads_q * w.batch / heads
+    return dict(value=w.batch / per_step, unit="decoded tokens/s", cores=_oracle_cores(),
+                kind="oracle",
+                sample=f"{heads} q heads of {w.name} at pos L-1 (selection of the last block + "
+                       f"fp64 decode attention), scaled to {w.heads_q} heads; {dt:.2f} s")
+
+
+def oracle_rows_sample(w: Workload, theta: float, what: str, n_rows: int = 64):
+    """fp64 oracle on the last `n_rows` rows of q head 0: FP8 (quantisation
+    + attention of the dequantised operands) or the key mass (LSE of each
+    row, then exp(s - LSE) over its kept set); TFLOP/s on 4 d (FP8) or 2 d
+    (key mass) per kept pair."""
+    from oracle import attention as oatt
+    from oracle import decode as odec
+    from oracle import fp8 as ofp8
+    from oracle import selection as osel
+    from workloads import bf16_bits_to_f32
+    inp = generate(w, kv_groups=[0])
+    L = w.seq_len
+    q32 = bf16_bits_to_f32(inp.q[0, 0])
+    k32 = bf16_bits_to_f32(inp.k[0, 0])
+    v32 = bf16_bits_to_f32(inp.v[0, 0])
+    rows = list(range(L - n_rows, L))
+    blocks = sorted({i // 128 for i in rows})
+    t0 = time.perf_counter()
+    qh, kh, vh = (x.astype(np.float64) for x in (q32, k32, v32))
+    sel = {qb: osel.anchor_block(qh, kh, qb, bq=128, sink=w.sink, local=w.local,
+                                 theta=theta).kept for qb in blocks}
+    keys_of = odec.prefill_keys_of_row(L, lambda b: sel[b], bq=128, sink=w.sink, local=w.local)
+    if what == "fp8":
+        q_hat, k_hat, v_hat = ofp8.dequantized_head(q32, k32, v32)
+        for i in rows:
+            oatt.attend_row(q_hat[i], k_hat, v_hat, keys_of(i), 1 / math.sqrt(128))
+        per_pair = 4 * 128
+    else:
+        _, lse = oatt.attend_rows(qh, kh, vh, rows, lambda i: i // 128, lambda b: sel[b], bq=128,
+                                  sink=w.sink, local=w.local)
+        odec.key_mass(qh[rows[0]:], kh, lse, range(len(rows)),
+                      lambda n: keys_of(rows[n]))
+        per_pair = 2 * 128
+    dt = time.perf_counter() - t0
+    pairs = sum(len(keys_of(i)) for i in rows)
+    return dict(value=per_pair * pairs / dt / 1e12, unit="TFLOP/s", cores=_oracle_cores(),
+                kind="oracle",
+                sample=f"q head 0, last {n_rows} rows of {w.name} ({what}); {dt:.2f} s")
 
 
 def variant_bench(args, w: Workload):
@@ -627,6 +705,7 @@ def variant_bench(args, w: Workload):
                                     + (" x 2 (nominal fp8:bf16)" if args.fp8 else "")},
         "clocks": clk.summary(),
         "gpu_launches": n_launch * args.steps,
+        "cpu_baseline": oracle_rows_sample(w, args.theta, "fp8" if args.fp8 else "key_mass"),
     }
     print(json.dumps(line), flush=True)
 
