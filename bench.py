@@ -506,7 +506,8 @@ def decode_bench(args, w: Workload):
     group = Hq // Hkv
     gh = next(d for d in range(8, 0, -1) if group % d == 0)
     units = B * Hkv * (group // gh)
-    counts = sc[:4 * units].view(torch.int32).cpu().numpy().astype(np.int64)
+    # the union counts follow the scratch's 256 reserved bytes (spa_decode.cu layout)
+    counts = sc[256:256 + 4 * units].view(torch.int32).cpu().numpy().astype(np.int64)
     qb = (L - 1) // 128
     ls = max(0, (qb + 1) * 128 - w.local)
     uk = w.block_k if args.mode == "sale" else 1

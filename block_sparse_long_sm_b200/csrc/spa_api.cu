@@ -37,8 +37,8 @@ Fp8Layout fp8_layout(const spa_params* p) {
   f.vs = f.ks + bkv;
   f.kmean = f.vs + bkv * 128;
   f.floats = f.kmean + bkv * 128;
-  f.kpart = 0;
-  f.kabs = align_up((size_t)bkv * kKmeanChunks * 128 * 8);
+  f.kpart = kHeaderBytes;      // reserved bytes first: every valid call has a non-zero size
+  f.kabs = align_up(f.kpart + (size_t)bkv * kKmeanChunks * 128 * 8);
   f.vabs = align_up(f.kabs + (size_t)bkv * 4);
   f.scratch = align_up(f.vabs + (size_t)bkv * 128 * 4);
   return f;

@@ -42,7 +42,8 @@ int chunks_for(long long units, long long keys_bound) {
   return (int)c;
 }
 
-// Scratch layout (byte offsets, each region 256-aligned): union counts
+// Scratch layout (byte offsets, each region 256-aligned): 256 reserved bytes
+// (so that every valid parameter set has a non-zero size); union counts
 // int32[units]; union lists uint32[units][union_stride]; tag words
 // uint32[units][union_stride / 4]; partials float[units][max_chunks][gh][132].
 DecodeLayout decode_layout(const spa_params* p, int kv_capacity) {
@@ -63,7 +64,7 @@ DecodeLayout decode_layout(const spa_params* p, int kv_capacity) {
   d.list_qb_off = cap_prefix(d.qb, 128, (long long)p->local + p->sink) / d.uk;
   d.union_stride = ((long long)d.cand_units + 3) / 4 * 4;
   d.max_chunks = chunks_for(d.units > 0 ? d.units : 1, kv_capacity);
-  size_t off = 0;
+  size_t off = kHeaderBytes;
   auto take = [&](size_t bytes) {
     const size_t at = off;
     off = align_up(off + bytes);
