@@ -238,6 +238,9 @@ def main():
     ap.add_argument("--window-tiles", action="store_true",
                     help="paired attention with contiguous masked windows for near-dense "
                          "selected keys (SPA_DEBUG_WINDOW_TILES)")
+    ap.add_argument("--sale-wide", action="store_true",
+                    help="SALE plan with the sixteen-warp block scan (SPA_DEBUG_SALE_WIDE), in "
+                         "the SALE leg of the extras and in --mode sale")
     ap.add_argument("--key-mass", action="store_true",
                     help="key mass from the prefill LSE over the plan instead of the headline step")
     args = ap.parse_args()
@@ -280,7 +283,8 @@ def main():
     o = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
     p = spa.make_params(B, Hq, Hkv, L, mode=args.mode, sink=w.sink, local=w.local,
                         theta=args.theta, tau=w.tau, block_k=w.block_k if args.mode == "sale" else None,
-                        debug_flags=spa.SPA_DEBUG_WINDOW_TILES if args.window_tiles else 0)
+                        debug_flags=(spa.SPA_DEBUG_WINDOW_TILES if args.window_tiles else 0) |
+                        (spa.SPA_DEBUG_SALE_WIDE if args.sale_wide else 0))
     ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
 
     def step():
@@ -756,14 +760,16 @@ def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, st
 
     # SALE mode
     ps = spa.make_params(B, Hq, Hkv, L, mode="sale", sink=w.sink, local=w.local, tau=w.tau,
-                         block_k=w.block_k)
+                         block_k=w.block_k,
+                         debug_flags=spa.SPA_DEBUG_SALE_WIDE if args.sale_wide else 0)
     wss = torch.empty(spa.sparse_prefill_workspace_bytes(ps), dtype=torch.uint8, device=dev)
     spa.check(spa.sparse_prefill_plan(ps, q, k, wss, stream=stream))
     sale_plan = timed(lambda: spa.check(spa.sparse_prefill_plan(ps, q, k, wss, stream=stream)))
     sale_attn = timed(lambda: spa.check(spa.sparse_prefill_attn(ps, q, k, v, wss, o, None, stream=stream)))
     st, ss = spa.sparse_prefill_stats(ps, wss, stream=stream)
     sflops = spa.kept_flops(ss)
-    out["sale"] = {"tau": w.tau, "block_k": w.block_k, "plan_ms": sale_plan, "attn_ms": sale_attn,
+    out["sale"] = {"tau": w.tau, "block_k": w.block_k, "scan": "wide" if args.sale_wide else "default",
+                   "plan_ms": sale_plan, "attn_ms": sale_attn,
                    "kept_fraction": ss.kept_pairs / ss.dense_pairs,
                    "kept_tflops": sflops / ((sale_plan + sale_attn) / 1e3) / 1e12}
     del wss
