@@ -203,3 +203,14 @@ def test_llama_128k_layer():
     dec = Decode(run, inp, L + 64, seed=23)
     for i, pos in enumerate((L - 1, L + 63)):
         dec.compare(_queries(1, w.heads_q, 600 + i, bias=0.5), pos, heads=heads)
+
+
+@pytest.mark.gpu_pending
+def test_batch_of_two():
+    L, cap = 1100, 1200
+    w = C0_TINY.with_(batch=2, heads_q=4, heads_kv=2, sink=64, local=256)
+    inp = generate(w, seq_len=L)
+    run = Run(inp, mode="anchor", sink=64, local=256, theta=2.5, do_attn=False)
+    dec = Decode(run, inp, cap, seed=29)
+    for i, pos in enumerate((L - 1, cap - 1)):
+        dec.compare(_queries(2, 4, 700 + i, bias=0.5), pos)

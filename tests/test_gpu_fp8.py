@@ -135,3 +135,14 @@ def test_fp8_llama_32k_sampled():
     for h in (0, 13, 31):
         _check_quantisation(fr, inp, 0, h)
         _check_outputs(fr, inp, 0, h, sample_rows(w.seq_len, 16, h, must=(0, 128, w.seq_len - 1)))
+
+
+def test_fp8_batch_of_two():
+    w = C0_TINY.with_(batch=2, heads_q=4, heads_kv=2, sink=64, local=256)
+    L = 900
+    inp = generate(w, seq_len=L)
+    run = Run(inp, mode="anchor", sink=64, local=256, theta=2.5, do_attn=False)
+    fr = Fp8Run(run)
+    for b in range(2):
+        _check_quantisation(fr, inp, b, 3)
+        _check_outputs(fr, inp, b, 3, list(range(0, L, 17)) + [L - 1])

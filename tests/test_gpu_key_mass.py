@@ -102,3 +102,12 @@ def test_key_mass_llama_32k_conserves_the_rows():
     want = run.group * w.seq_len
     assert np.all(np.abs(per_kv - want) <= (REL + math.expm1(2e-3)) * want), per_kv
     assert np.all(got >= 0)
+
+
+def test_key_mass_batch_of_two():
+    w = C0_TINY.with_(batch=2, heads_q=4, heads_kv=2, sink=64, local=256)
+    inp = generate(w, seq_len=700)
+    run = Run(inp, mode="anchor", sink=64, local=256, theta=2.5)
+    ref, lse = _oracle(run, inp, 0)
+    got = _gpu_mass(run, torch.from_numpy(lse.astype(np.float32)).cuda(), 0)
+    assert np.all(np.abs(got - ref) <= REL * ref + 1e-6)

@@ -55,3 +55,10 @@ def test_window_tiles_llama_32k():
     rows = {(0, h): sample_rows(w.seq_len, 24, h, must=(0, 127, 128, w.seq_len - 1))
             for h in (0, 1, 17, 30)}
     compare_outputs(run, inp, rows)
+
+
+def test_window_tiles_batch_of_two():
+    w = C0_TINY.with_(batch=2, heads_q=4, heads_kv=2)
+    inp = generate(w, seq_len=1500)
+    run = Run(inp, mode="anchor", sink=w.sink, local=w.local, theta=4.0, debug_flags=WIN)
+    compare_outputs(run, inp, {(b, h): range(1500) for b in range(2) for h in (0, 3)})
