@@ -146,3 +146,16 @@ def test_fp8_batch_of_two():
     for b in range(2):
         _check_quantisation(fr, inp, b, 3)
         _check_outputs(fr, inp, b, 3, list(range(0, L, 17)) + [L - 1])
+
+
+def test_fp8_diffuse_heads():
+    # attention spread thinly over many keys (no sink bias): the regime where
+    # the E4M3 rounding of many small probabilities matters most
+    w = C0_TINY.with_(heads_q=4, heads_kv=2, sink=64, local=256, diffuse_kv_heads=(0, 1))
+    L = 1200
+    inp = generate(w, seq_len=L)
+    run = Run(inp, mode="anchor", sink=64, local=256, theta=1.0, do_attn=False)
+    fr = Fp8Run(run)
+    for h in (0, 2):
+        _check_quantisation(fr, inp, 0, h)
+        _check_outputs(fr, inp, 0, h, list(range(0, L, 11)) + [L - 1])
