@@ -11,8 +11,11 @@
 // copies per operand, and the keys not in the union are masked column by
 // column through the per-head membership masks the producer already
 // publishes; otherwise the next 128 union keys are gathered as before.
-// Attention over a key set does not depend on the order of its tiles, so the
-// result is the paired kernel's up to rounding.
+// When both heads keep every candidate of the block (the near-dense case: at
+// theta = 5 on the 128K layer every block), the selected keys are simply
+// [sink, ls) and go as plain contiguous tiles without reading the list at
+// all.  Attention over a key set does not depend on the order of its tiles,
+// so the result is the paired kernel's up to rounding.
 //
 // The number of selected tiles now depends on the keys.  Rather than count
 // them up front (a chain of dependent list reads), the producer publishes for
@@ -163,7 +166,13 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
     uint32_t ntg[4] = {0u, 0u, 0u, 0u};
     int n_cur = 0;                             // union ordinal of the next selected tile
     int loc = 0;                               // local tiles issued
-    if (n_total > 0) fetch_at(0, nj, ntg);
+    // both heads keep every candidate (the union has every candidate and the
+    // two lists never differ: the shared prefix is the whole union), so the
+    // selected keys are [sink, ls), loaded as plain contiguous tiles without
+    // reading the list
+    const bool all_kept = n_total > 0 && n_total == max(0, it.ls - a.sink) &&
+                          pi.split * a.list_unit >= n_total;
+    if (n_total > 0 && !all_kept) fetch_at(0, nj, ntg);
     for (int t = 0;; ++t) {
       const int ks = t % kPairKStages, vs = t % kPairVStages;
       if (t >= kPairKStages &&
@@ -181,6 +190,12 @@ sparse_attn_pair_win_kernel(const __grid_constant__ CUtensorMap tm_q,
         td.key0 = t * 128;
         td.valid = min(128, it.sink_end - td.key0);
         td.causal = 0;
+      } else if (n_cur < n_total && all_kept) {
+        td.gather = 0;
+        td.key0 = a.sink + n_cur;
+        td.valid = min(128, n_total - n_cur);
+        td.causal = 0;
+        n_cur += td.valid;
       } else if (n_cur < n_total) {
         td.gather = 1;
         td.key0 = 0;

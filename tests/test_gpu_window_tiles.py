@@ -4,7 +4,8 @@ are loaded contiguously with the absent keys masked, the rest gathered.  The
 attention is over the same kept sets as the default paired kernel, so the
 same stated bounds hold against the oracle on the GPU's own kept sets.
 
-Densities from near-dense (every window tile) through mixed to sparse
+Densities from every candidate kept by both heads (the contiguous fast
+path, no list read) and near-dense (window tiles) through mixed to sparse
 (every tile gathered), ragged lengths, SALE key blocks and step groups.
 
 These tests carry the ``gpu_pending`` marker until their first passing run
@@ -23,7 +24,7 @@ pytestmark = pytest.mark.gpu_pending
 WIN = spa.SPA_DEBUG_WINDOW_TILES
 
 
-@pytest.mark.parametrize("theta", [7.0, 5.0, 4.0, 3.0, 2.0])
+@pytest.mark.parametrize("theta", [float("inf"), 7.0, 5.0, 4.0, 3.0, 2.0])
 def test_window_tiles_all_rows(theta):
     w = C0_TINY.with_(heads_q=2, heads_kv=1)
     inp = generate(w)
