@@ -162,13 +162,24 @@ key_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
         }
         if (bad) atomicOr(a.err, kErrBadIndex);
+        // 128 consecutive keys (a near-dense selection): two tiled copies
+        const int last = __shfl_sync(0xffffffffu, j[3], 31);
+        const bool contiguous = td.valid == 128 && last - first == 127 && first >= 0 &&
+                                last < a.g.L;
         if (lane == 0) mbar_arrive_expect_tx(kf, kTileBytes);
         __syncwarp();
-        const uint32_t roff = lane * 4u * 128u;
-        tma_gather4(s_k(st) + roff, &tm_kg, kf, 0, kv_row0 + j[0], kv_row0 + j[1],
-                    kv_row0 + j[2], kv_row0 + j[3]);
-        tma_gather4(s_k(st) + kHalfBytes + roff, &tm_kg, kf, 64, kv_row0 + j[0],
-                    kv_row0 + j[1], kv_row0 + j[2], kv_row0 + j[3]);
+        if (contiguous) {
+          if (lane == 0) {
+            tma_load_2d(s_k(st), &tm_k, kf, 0, kv_row0 + first);
+            tma_load_2d(s_k(st) + kHalfBytes, &tm_k, kf, 64, kv_row0 + first);
+          }
+        } else {
+          const uint32_t roff = lane * 4u * 128u;
+          tma_gather4(s_k(st) + roff, &tm_kg, kf, 0, kv_row0 + j[0], kv_row0 + j[1],
+                      kv_row0 + j[2], kv_row0 + j[3]);
+          tma_gather4(s_k(st) + kHalfBytes + roff, &tm_kg, kf, 64, kv_row0 + j[0],
+                      kv_row0 + j[1], kv_row0 + j[2], kv_row0 + j[3]);
+        }
       }
       issued = t + 1;
     }
