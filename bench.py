@@ -506,20 +506,34 @@ def decode_bench(args, w: Workload):
     st, _ = spa.sparse_prefill_stats(p, ws, stream=stream)
     spa.check(st, "stats")
 
-    # key-set sizes per (b, kv head, subgroup) from the prepared union counts
+    # key-set sizes per (b, kv head, subgroup of up to 8 q heads): the union
+    # of the last prompt block's selections, read from the plan's lists
+    from block_sparse_long_sm_b200.binding import WorkspaceView
+    view = WorkspaceView(p, ws)
+    counts_h = view.counts.cpu().numpy()
     group = Hq // Hkv
     gh = next(d for d in range(8, 0, -1) if group % d == 0)
-    units = B * Hkv * (group // gh)
-    # the union counts follow the scratch's 256 reserved bytes (spa_decode.cu layout)
-    counts = sc[256:256 + 4 * units].view(torch.int32).cpu().numpy().astype(np.int64)
     qb = (L - 1) // 128
+    union_sizes = []
+    for b in range(B):
+        for g in range(Hkv):
+            for hs in range(group // gh):
+                sel = [np.zeros(0, np.int64)]
+                for j in range(gh):
+                    h = g * group + hs * gh + j
+                    if args.mode != "dense":   # only this block's list leaves the GPU
+                        n = int(counts_h[view.block_index(b, h, qb)])
+                        off = view.list_offset(b, h, qb)
+                        sel.append(view.lists[off:off + n].cpu().numpy().astype(np.int64))
+                union_sizes.append(len(np.unique(np.concatenate(sel))))
+    counts = np.array(union_sizes, dtype=np.int64)
     ls = max(0, (qb + 1) * 128 - w.local)
     uk = w.block_k if args.mode == "sale" else 1
     bytes_steps = []
     for i in range(args.steps):
         pos = L - 1 + warm + i
         if args.mode == "dense":
-            keys = units * (pos + 1)
+            keys = len(counts) * (pos + 1)
         else:
             s1 = min(w.sink, pos + 1)
             keys = int(np.sum(s1 + counts * uk + (pos + 1 - max(ls, s1))))
