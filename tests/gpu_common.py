@@ -235,3 +235,40 @@ def edge_blocks(L: int, extra: int, seed: int) -> List[int]:
     s = {0, 1, 2, 3, nqb // 2, nqb - 2, nqb - 1}
     s.update(int(x) for x in rng.integers(0, nqb, size=extra))
     return sorted(x for x in s if 0 <= x < nqb)
+
+
+def sale_scratch(run: Run) -> Dict[str, np.ndarray]:
+    """The SALE plan's quantised operands, read back from the workspace.
+
+    Offsets follow the workspace layout of SALE mode: after the header, the
+    counts and the lists come the fp64 K-mean partial sums (64 chunks x 128
+    per (b, kv head)), the fp32 K mean [B*Hkv][128], the int8 Q codes
+    [B*Hq][L][128], the int8 K codes [B*Hkv][L][128], the fp32 Q scales
+    [B*Hq*nqb] and the fp32 K scales [B*Hkv][nkb]; every region starts on a
+    256-byte boundary.
+    """
+    p = run.params
+    assert p.mode == spa.SPA_MODE_SALE
+    B, Hq, Hkv, L, bk = run.B, run.Hq, run.Hkv, run.L, p.block_k
+    nqb, nkb = (L + 127) // 128, (L + bk - 1) // bk
+    view = run.view
+    a = lambda x: (x + 255) // 256 * 256
+    off = a(256 + 4 * view.nb)                       # lists
+    off = a(off + 4 * B * Hq * view.per_head)        # K-mean partials
+    off = a(off + B * Hkv * 64 * 128 * 8)            # K mean
+    kmean_at = off
+    off = a(off + B * Hkv * 128 * 4)
+    q8_at = off
+    off = a(off + B * Hq * L * 128)
+    k8_at = off
+    off = a(off + B * Hkv * L * 128)
+    sq_at = off
+    off = a(off + view.nb * 4)
+    sk_at = off
+    ws = run.ws.cpu().numpy()
+    take = lambda at, n, dt: ws[at:at + n * np.dtype(dt).itemsize].view(dt)
+    return dict(kmean=take(kmean_at, B * Hkv * 128, np.float32).reshape(B, Hkv, 128),
+                qcodes=take(q8_at, B * Hq * L * 128, np.int8).reshape(B, Hq, L, 128),
+                kcodes=take(k8_at, B * Hkv * L * 128, np.int8).reshape(B, Hkv, L, 128),
+                qscales=take(sq_at, view.nb, np.float32).reshape(B, Hq, nqb),
+                kscales=take(sk_at, B * Hkv * nkb, np.float32).reshape(B, Hkv, nkb))

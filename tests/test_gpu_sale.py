@@ -22,22 +22,30 @@ def test_sale_small_all_blocks(L, tau, bk, sink):
     compare_outputs(run, inp, {(0, 0): range(L)})
 
 
-def test_sale_quantisation_codes_bit_exact():
-    """The int4 codes and scales in the workspace equal the oracle's (fp32 decisions)."""
-    import torch
+@pytest.mark.parametrize("B,hq,hkv,L,bk", [(1, 1, 1, 2048, 32), (1, 4, 2, 1900, 16),
+                                            (2, 2, 1, 1000, 64)])
+def test_sale_quantisation_codes_bit_exact(B, hq, hkv, L, bk):
+    """The int4 codes, their fp32 scales and the fp32 K mean that the plan
+    leaves in the workspace equal the oracle's, bit for bit (the quantisation
+    step is fp32 on both sides; the K sum is exact in fp64 for bf16 keys)."""
     from oracle import selection as osel
-    w = C0_TINY.with_(sink=64, local=256)
-    L = 2048
+    from gpu_common import sale_scratch
+    w = C0_TINY.with_(batch=B, heads_q=hq, heads_kv=hkv, sink=64, local=256)
     inp = generate(w, seq_len=L)
-    run = Run(inp, mode="sale", sink=64, local=256, tau=1e-3, block_k=32, do_attn=False)
-    prep = osel.sale_prepare(bf16_bits_to_f32(inp.q[0, 0]), bf16_bits_to_f32(inp.k[0, 0]),
-                             bq=128, bk=32)
-    # codes are observable through the selection only; check the selection on all blocks
-    # (bit-exact away from near-ties) and the kept counts in the stats
-    res = compare_sale_masks(run, inp, [(0, 0)])
-    assert run.stats.kept_candidates == int(run.counts.sum()) * 32
-    assert res["blocks"] == (L + 127) // 128
-    assert prep.qcodes.shape == (L, 128)
+    run = Run(inp, mode="sale", sink=64, local=256, tau=1e-3, block_k=bk, do_attn=False)
+    got = sale_scratch(run)
+    for b in range(B):
+        for h in range(hq):
+            g = h // (hq // hkv)
+            prep = osel.sale_prepare(bf16_bits_to_f32(inp.q[b, h]), bf16_bits_to_f32(inp.k[b, g]),
+                                     bq=128, bk=bk)
+            np.testing.assert_array_equal(got["qcodes"][b, h], prep.qcodes)
+            np.testing.assert_array_equal(got["qscales"][b, h], prep.qscales)
+            np.testing.assert_array_equal(got["kcodes"][b, g], prep.kcodes)
+            np.testing.assert_array_equal(got["kscales"][b, g], prep.kscales)
+            np.testing.assert_array_equal(got["kmean"][b, g], prep.kmean)
+    # the selection built on them, bit-exact away from near-ties
+    compare_sale_masks(run, inp, [(b, h) for b in range(B) for h in range(hq)])
 
 
 def test_sale_c2_shape_16k_two_heads_all_blocks():

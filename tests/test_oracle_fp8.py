@@ -115,3 +115,12 @@ def test_dequantised_operands_within_half_a_step():
         assert np.all(np.abs(x - xh) <= bound)
         # the largest magnitude of each scaling group maps to exactly 448
     assert np.max(np.abs(q_hat[:128])) == np.float64(qs[0]) * 448.0
+
+
+def test_smoothing_mean_is_the_exact_mean_rounded_once():
+    # the same exact-fraction fixture as the int4 estimate's: smooth_k must
+    # subtract the correctly rounded fp32 mean (an fp32 sum, or a sum rounded
+    # to fp32 before the division, gives other values on these keys)
+    from test_oracle_sale import exact_mean_fixture
+    k, want = exact_mean_fixture(seed=12, L=2999, d=64)
+    np.testing.assert_array_equal(fp8.smooth_k(k), (k - want).astype(np.float32))

@@ -97,6 +97,19 @@ CASES = [
     ("sale_quant_step", osel, "_quantize_rows_fp32", "seven = np.float32(7.0)",
      "seven = np.float32(8.0)", [t_sale.test_integer_inputs_quantise_exactly,
                                  t_sale.test_quantisation_properties_on_generated_data]),
+    # SALE smoothing mean: summed in fp64 (not fp32) ...
+    ("sale_mean_fp32_sum", osel, "sale_smooth_mean", "kh32.astype(np.float64).sum(axis=0)",
+     "kh32.astype(np.float32).sum(axis=0, dtype=np.float32)",
+     [t_sale.test_smoothing_mean_is_the_exact_mean_rounded_once]),
+    # ... and rounded to fp32 once, after the division
+    ("sale_mean_rounded_before_division", osel, "sale_smooth_mean",
+     "(kh32.astype(np.float64).sum(axis=0) / float(L)).astype(np.float32)",
+     "kh32.astype(np.float64).sum(axis=0).astype(np.float32) / np.float32(L)",
+     [t_sale.test_smoothing_mean_is_the_exact_mean_rounded_once]),
+    # FP8 smoothing: the same mean reading
+    ("fp8_mean_fp32_sum", ofp8, "smooth_k", "kh32.astype(np.float64).sum(axis=0)",
+     "kh32.astype(np.float32).sum(axis=0, dtype=np.float32)",
+     [t_fp8.test_smoothing_mean_is_the_exact_mean_rounded_once]),
     # a block is kept when its largest relative score reaches tau
     ("sale_block_min", osel, "sale_block", "margin = excess.reshape(-1, bk).max(axis=1)",
      "margin = excess.reshape(-1, bk).min(axis=1)", [t_sale.test_handmade_sale_cases,

@@ -11,11 +11,17 @@
 * A hand-derived example (tests/golden/sale_handmade.json) fixes em/el over
   the sink-local area, the threshold, the block maximum and tie handling.
 * Nesting in tau.
+* The smoothing mean (the per-head K mean over the sequence) equals the
+  correctly rounded fp32 value of the exact rational mean, computed here with
+  exact fractions, on bf16-valued keys with a non-zero mean and a length that
+  is not a power of two -- inputs on which an fp32 sum, or rounding the sum
+  to fp32 before dividing, lands on a different fp32 value.
 """
 
 import json
 import math
 import os
+from fractions import Fraction
 
 import numpy as np
 import pytest
@@ -159,3 +165,50 @@ def test_tiny_tau_keeps_every_candidate_block():
                              bq=128, bk=32)
     r = osel.sale_block(prep, 6, L=1024, bq=128, bk=32, sink=64, local=128, tau=1e-300)
     np.testing.assert_array_equal(r.kept_blocks, r.cand_blocks)
+
+
+def _bf16_valued(x: np.ndarray) -> np.ndarray:
+    """Round fp32 values to bf16 (nearest even) and return them as fp32."""
+    b = x.astype(np.float32).view(np.uint32).astype(np.uint64)
+    b = ((b + 0x7FFF + ((b >> 16) & 1)) >> 16) << 16
+    return b.astype(np.uint32).view(np.float32)
+
+
+def _nearest_fp32(fr: Fraction) -> np.float32:
+    """The fp32 value nearest to an exact rational (no ties allowed here)."""
+    f = np.float32(float(fr))
+    cands = [np.nextafter(f, np.float32(-np.inf)), f, np.nextafter(f, np.float32(np.inf))]
+    dist = sorted((abs(Fraction(float(c)) - fr), n) for n, c in enumerate(cands))
+    assert dist[0][0] != dist[1][0], "the fixture must avoid an fp32 tie"
+    # the mean is rounded twice (fp64 division, then fp32): a result within
+    # 2^-50 (relative) of an fp32 midpoint could round either way
+    half_gap = abs(Fraction(float(cands[2])) - Fraction(float(cands[1]))) / 2
+    assert abs(dist[0][0] - half_gap) > abs(fr) * Fraction(1, 2 ** 50)
+    return cands[dist[0][1]]
+
+
+def exact_mean_fixture(seed: int = 11, L: int = 3000, d: int = 128):
+    """bf16-valued keys with a non-zero mean, and their exact per-column means
+    rounded once to fp32."""
+    rng = np.random.default_rng(seed)
+    k = _bf16_valued(rng.normal(0, 1, (L, d)).astype(np.float32) + np.float32(2.5))
+    want = np.array([_nearest_fp32(sum(Fraction(float(v)) for v in k[:, c]) / L)
+                     for c in range(d)], dtype=np.float32)
+    return k, want
+
+
+def test_smoothing_mean_is_the_exact_mean_rounded_once():
+    k, want = exact_mean_fixture()
+    L = k.shape[0]
+    # the fixture separates the reading from its plausible slips
+    assert np.count_nonzero(k.sum(axis=0, dtype=np.float32) / np.float32(L) != want) > 0
+    assert np.count_nonzero(k.astype(np.float64).sum(axis=0).astype(np.float32) /
+                            np.float32(L) != want) > 0
+    np.testing.assert_array_equal(osel.sale_smooth_mean(k), want)
+    # and the smoothed keys the codes are taken from are K minus that mean (fp32)
+    codes, scales, mean = osel.sale_quantize_k(k, 32)
+    np.testing.assert_array_equal(mean, want)
+    for blk in range(L // 32):
+        ks = k[blk * 32:(blk + 1) * 32] - want
+        amax = np.float32(np.abs(ks).max())
+        assert scales[blk] == np.float32(amax / np.float32(7.0))
