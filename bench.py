@@ -238,9 +238,6 @@ def main():
     ap.add_argument("--window-tiles", action="store_true",
                     help="paired attention with contiguous masked windows for near-dense "
                          "selected keys (SPA_DEBUG_WINDOW_TILES)")
-    ap.add_argument("--sale-wide", action="store_true",
-                    help="SALE plan with the sixteen-warp block scan (SPA_DEBUG_SALE_WIDE), in "
-                         "the SALE leg of the extras and in --mode sale")
     ap.add_argument("--key-mass", action="store_true",
                     help="key mass from the prefill LSE over the plan instead of the headline step")
     args = ap.parse_args()
@@ -283,8 +280,7 @@ def main():
     o = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
     p = spa.make_params(B, Hq, Hkv, L, mode=args.mode, sink=w.sink, local=w.local,
                         theta=args.theta, tau=w.tau, block_k=w.block_k if args.mode == "sale" else None,
-                        debug_flags=(spa.SPA_DEBUG_WINDOW_TILES if args.window_tiles else 0) |
-                        (spa.SPA_DEBUG_SALE_WIDE if args.sale_wide else 0))
+                        debug_flags=(spa.SPA_DEBUG_WINDOW_TILES if args.window_tiles else 0))
     ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
 
     def step():
@@ -729,6 +725,36 @@ def variant_bench(args, w: Workload):
     print(json.dumps(line), flush=True)
 
 
+# SALE thresholds that really skip key blocks on the synthetic 128K layer
+# (the oracle keeps about 46 % of the candidate blocks at 0.1)
+SALE_PRUNING_TAUS = (0.1,)
+
+
+def _operating_point(spa, torch, timed, p, ws, q, k, v, o, stream, peaks, dense_ms, label):
+    """Plan and attention of one selection setting on the resident layer:
+    kept fraction, times, kept-FLOP roofline of the attention, selection
+    bytes against HBM, and the speedup over the same kernel run dense."""
+    spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream))
+    spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None, stream=stream))
+    plan_ms = timed(lambda: spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream)))
+    attn_ms = timed(lambda: spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None,
+                                                              stream=stream)))
+    st, s = spa.sparse_prefill_stats(p, ws, stream=stream)
+    spa.check(st, "stats")
+    flops = spa.kept_flops(s)
+    B, Hq, Hkv, L = p.batch, p.heads_q, p.heads_kv, p.seq_len
+    unit = p.block_k if p.mode == spa.SPA_MODE_SALE else 1
+    alg_bytes = 2 * B * Hq * L * 128 + 2 * B * Hkv * L * 128 + 4 * s.kept_candidates // unit
+    tfl = flops / (attn_ms / 1e3) / 1e12
+    return dict(label, kept_fraction=s.kept_pairs / s.dense_pairs,
+                kept_candidates_fraction=s.kept_candidates / max(1, s.candidates),
+                plan_ms=plan_ms, attn_ms=attn_ms, step_ms=plan_ms + attn_ms,
+                attn_tflops=tfl, attn_frac=tfl / peaks["bf16_sus"],
+                selection_gbs=alg_bytes / (plan_ms / 1e3) / 1e9,
+                selection_frac=alg_bytes / (plan_ms / 1e3) / 1e9 / peaks["hbm"],
+                speedup_vs_dense=dense_ms / (plan_ms + attn_ms))
+
+
 def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, stats):
     """Selection roofline, SALE mode, dense mode, end-to-end and the CPU baseline."""
     peaks = _peaks()
@@ -747,6 +773,17 @@ def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, st
             ts.append(a.elapsed_time(b))
         return statistics.median(ts)
 
+    # dense mode: same attention kernel over every causal key
+    pd = spa.make_params(B, Hq, Hkv, L, mode="dense", sink=w.sink, local=w.local)
+    wsd = torch.empty(spa.sparse_prefill_workspace_bytes(pd), dtype=torch.uint8, device=dev)
+    spa.check(spa.sparse_prefill_plan(pd, q, k, wsd, stream=stream))
+    dense_ms = timed(lambda: spa.check(spa.sparse_prefill_attn(pd, q, k, v, wsd, o, None, stream=stream)))
+    st, sd = spa.sparse_prefill_stats(pd, wsd, stream=stream)
+    dflops = spa.kept_flops(sd)
+    out["dense"] = {"attn_ms": dense_ms, "tflops": dflops / (dense_ms / 1e3) / 1e12,
+                    "frac": dflops / (dense_ms / 1e3) / 1e12 / peaks["bf16_sus"]}
+    del wsd
+
     # selection roofline (anchor plan): algorithmic bytes = read Q + read K once + write lists
     p = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=w.sink, local=w.local, theta=args.theta)
     ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
@@ -761,29 +798,35 @@ def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, st
                         "candidates": s.candidates}
     del ws
 
-    # dense mode: same attention kernel over every causal key
-    pd = spa.make_params(B, Hq, Hkv, L, mode="dense", sink=w.sink, local=w.local)
-    wsd = torch.empty(spa.sparse_prefill_workspace_bytes(pd), dtype=torch.uint8, device=dev)
-    spa.check(spa.sparse_prefill_plan(pd, q, k, wsd, stream=stream))
-    dense_ms = timed(lambda: spa.check(spa.sparse_prefill_attn(pd, q, k, v, wsd, o, None, stream=stream)))
-    st, sd = spa.sparse_prefill_stats(pd, wsd, stream=stream)
-    dflops = spa.kept_flops(sd)
-    out["dense"] = {"attn_ms": dense_ms, "tflops": dflops / (dense_ms / 1e3) / 1e12,
-                    "frac": dflops / (dense_ms / 1e3) / 1e12 / peaks["bf16_sus"]}
-    del wsd
+    # the sparse operating points of the same layer: theta swept over {3, 7}
+    # besides the headline's value, and SALE at a tau that skips key blocks
+    points = []
+    for theta in (3.0, 7.0):
+        pt = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=w.sink, local=w.local, theta=theta,
+                             debug_flags=spa.SPA_DEBUG_WINDOW_TILES if args.window_tiles else 0)
+        wst = torch.empty(spa.sparse_prefill_workspace_bytes(pt), dtype=torch.uint8, device=dev)
+        points.append(_operating_point(spa, torch, timed, pt, wst, q, k, v, o, stream, peaks,
+                                       dense_ms, dict(mode="anchor", theta=theta)))
+        del wst
+    for tau in SALE_PRUNING_TAUS:
+        pt = spa.make_params(B, Hq, Hkv, L, mode="sale", sink=w.sink, local=w.local, tau=tau,
+                             block_k=w.block_k)
+        wst = torch.empty(spa.sparse_prefill_workspace_bytes(pt), dtype=torch.uint8, device=dev)
+        points.append(_operating_point(spa, torch, timed, pt, wst, q, k, v, o, stream, peaks,
+                                       dense_ms, dict(mode="sale", tau=tau, block_k=w.block_k)))
+        del wst
+    out["operating_points"] = points
 
     # SALE mode
     ps = spa.make_params(B, Hq, Hkv, L, mode="sale", sink=w.sink, local=w.local, tau=w.tau,
-                         block_k=w.block_k,
-                         debug_flags=spa.SPA_DEBUG_SALE_WIDE if args.sale_wide else 0)
+                         block_k=w.block_k)
     wss = torch.empty(spa.sparse_prefill_workspace_bytes(ps), dtype=torch.uint8, device=dev)
     spa.check(spa.sparse_prefill_plan(ps, q, k, wss, stream=stream))
     sale_plan = timed(lambda: spa.check(spa.sparse_prefill_plan(ps, q, k, wss, stream=stream)))
     sale_attn = timed(lambda: spa.check(spa.sparse_prefill_attn(ps, q, k, v, wss, o, None, stream=stream)))
     st, ss = spa.sparse_prefill_stats(ps, wss, stream=stream)
     sflops = spa.kept_flops(ss)
-    out["sale"] = {"tau": w.tau, "block_k": w.block_k, "scan": "wide" if args.sale_wide else "default",
-                   "plan_ms": sale_plan, "attn_ms": sale_attn,
+    out["sale"] = {"tau": w.tau, "block_k": w.block_k, "plan_ms": sale_plan, "attn_ms": sale_attn,
                    "kept_fraction": ss.kept_pairs / ss.dense_pairs,
                    "kept_tflops": sflops / ((sale_plan + sale_attn) / 1e3) / 1e12}
     del wss

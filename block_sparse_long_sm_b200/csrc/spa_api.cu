@@ -16,7 +16,6 @@
 #include "host.cuh"
 #include "ptx.cuh"
 #include "sale.cuh"
-#include "sale_wide.cuh"
 #include "select.cuh"
 
 namespace {
@@ -158,15 +157,9 @@ SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const
                 reinterpret_cast<uint32_t*>(ws + lo.mask), lo.nwords, err, wait_ns(p), {}};
     for (int h = 0; h < Hq && h < SPA_MAX_TAU_HEADS; ++h)
       sa.tau_h[h] = p->tau_per_head ? p->tau_per_head[h] : p->tau;
-    if (p->debug_flags & SPA_DEBUG_SALE_WIDE) {
-      if (set_smem(sale_scan_wide_kernel, kSaleSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
-      sale_scan_wide_kernel<<<(unsigned)(BKV * lo.nqb * chunks), kSaleWideThreads, kSaleSmemBytes,
-                              stream>>>(tq8, tk8, sa);
-    } else {
-      if (set_smem(sale_scan_kernel, kSaleSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
-      sale_scan_kernel<<<(unsigned)(BKV * lo.nqb * chunks), kSaleThreads, kSaleSmemBytes,
-                         stream>>>(tq8, tk8, sa);
-    }
+    if (set_smem(sale_scan_kernel, kSaleSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
+    sale_scan_kernel<<<(unsigned)(BKV * lo.nqb * chunks), kSaleThreads, kSaleSmemBytes, stream>>>(
+        tq8, tk8, sa);
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   }
   if (lo.paired) {

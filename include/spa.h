@@ -125,11 +125,6 @@ typedef struct {
  * tile of 128 selected keys row by row.  Same result up to rounding. */
 #define SPA_DEBUG_WINDOW_TILES 0x2u
 
-/* Variant switch (SALE plan): the block scan with sixteen epilogue warps, one
- * head's TMEM lane quadrant each, instead of eight warps reading two heads in
- * turn.  Same result. */
-#define SPA_DEBUG_SALE_WIDE 0x4u
-
 typedef struct {
   uint32_t error_bits;       /* device error word: bit0 timeout, bit1 bad index */
   uint32_t reserved;

@@ -17,10 +17,6 @@ head subgroups), ANCHOR, SALE and DENSE, positions from L - 1 (where the
 decode key set is the last prompt row's prefill key set) to the end of the
 cache, a prompt of one token, a sink that covers the whole candidate range,
 repeated calls after one prepare, and the 128K Llama layer.
-
-Tests marked ``gpu_pending`` have not yet passed on a B200 and join the
-``gpu`` set after their first passing run (``pytest -m gpu_pending`` selects
-them).
 """
 
 import numpy as np
@@ -160,7 +156,7 @@ def test_dense_mode():
     dec.compare(_queries(1, 4, 301), cap - 1)
 
 
-@pytest.mark.gpu_pending
+@pytest.mark.gpu
 @pytest.mark.parametrize("L,sink,local,positions", [
     (1, 64, 128, (0, 1, 3)),          # one-token prompt: no candidates
     (300, 256, 128, (299, 310)),      # sink covers the candidate range
@@ -176,7 +172,7 @@ def test_degenerate_geometry(L, sink, local, positions):
         dec.compare(_queries(1, 2, 400 + i), pos)
 
 
-@pytest.mark.gpu_pending
+@pytest.mark.gpu
 def test_repeated_calls_are_identical():
     L, cap = 1200, 1300
     w = C0_TINY.with_(heads_q=4, heads_kv=2, sink=64, local=256)
@@ -191,7 +187,7 @@ def test_repeated_calls_are_identical():
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
-@pytest.mark.gpu_pending
+@pytest.mark.gpu
 def test_llama_128k_layer():
     w = C2_LLAMA_128K
     L = w.seq_len
@@ -205,7 +201,7 @@ def test_llama_128k_layer():
         dec.compare(_queries(1, w.heads_q, 600 + i, bias=0.5), pos, heads=heads)
 
 
-@pytest.mark.gpu_pending
+@pytest.mark.gpu
 def test_batch_of_two():
     L, cap = 1100, 1200
     w = C0_TINY.with_(batch=2, heads_q=4, heads_kv=2, sink=64, local=256)

@@ -9,9 +9,6 @@ Computation Pass on quantised operands, SageAttention-style).
   the bound of the kernel's arithmetic: the probabilities enter the PV product
   rounded to E4M3 (relative error <= 2^-4 each) and O is rounded to bf16, so
   |dO| <= 2^-4 (sum_j p_j |v^_j|) / l + 2^-8 |O| + 1e-4; LSE within 2e-3.
-
-These tests carry the ``gpu_pending`` marker until their first passing run
-on a B200 (``pytest -m gpu_pending``).
 """
 
 import numpy as np
@@ -25,7 +22,7 @@ from workloads import C0_TINY, bf16_bits_to_f32, generate
 
 from gpu_common import LSE_ABS, Run
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 E4M3_VALUES = np.array([ofp8.e4m3_decode(c) for c in range(256)])
 

@@ -10,9 +10,6 @@ sums as a bf16 probability (relative error <= 2^-8) and the sums are
 accumulated in fp32, so |d mass_j| <= (2^-8 + 2^-12) mass_j + 1e-6; with the
 attention kernel's own LSE (within 2e-3) the relative part grows by
 exp(2e-3) - 1.
-
-These tests carry the ``gpu_pending`` marker until their first passing run
-on a B200 (``pytest -m gpu_pending``).
 """
 
 import math
@@ -28,7 +25,7 @@ from workloads import C0_TINY, generate
 
 from gpu_common import Run, head_f64
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 REL = 2.0 ** -8 + 2.0 ** -12
 
