@@ -202,8 +202,14 @@ sparse_attn_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         }
         if (bad) atomicOr(a.err, kErrBadIndex);
         const int last = __shfl_sync(0xffffffffu, j[3], 31);
+        // 128 consecutive keys: every lane's four keys are exactly the next
+        // ones (a list entry out of order or repeated keeps the gather path)
         const bool contiguous = (td.valid == 128) && (last - first == 127) && first >= 0 &&
-                                first < a.g.L && last < a.g.L;
+                                first < a.g.L && last < a.g.L &&
+                                __all_sync(0xffffffffu, j[0] == first + 4 * lane &&
+                                                            j[1] == first + 4 * lane + 1 &&
+                                                            j[2] == first + 4 * lane + 2 &&
+                                                            j[3] == first + 4 * lane + 3);
         if (lane == 0) {
           mbar_arrive_expect_tx(kf, kTile8);
           mbar_arrive_expect_tx(vf, kTile8);

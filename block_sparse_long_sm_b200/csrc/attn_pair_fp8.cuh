@@ -219,7 +219,12 @@ sparse_attn_pair_fp8_kernel(const __grid_constant__ CUtensorMap tm_q,
         if (lane == 0) mbar_arrive(bar_tag0 + 8u * vs);   // publishes this tile's masks
         const int first = __shfl_sync(0xffffffffu, j[0], 0);
         const int last = __shfl_sync(0xffffffffu, j[3], 31);
-        contiguous = (td.valid == 128) && (last - first == 127);
+        // 128 consecutive keys: every lane's four keys are exactly the next
+        // ones (a list entry out of order or repeated keeps the gather path)
+        contiguous = (td.valid == 128) && (last - first == 127) &&
+                     __all_sync(0xffffffffu, j[0] == first + 4 * lane && j[1] == first + 4 * lane + 1 &&
+                                                 j[2] == first + 4 * lane + 2 &&
+                                                 j[3] == first + 4 * lane + 3);
         key0 = first;
       }
       if (lane == 0) {

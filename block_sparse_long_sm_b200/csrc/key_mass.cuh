@@ -164,8 +164,14 @@ key_mass_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (bad) atomicOr(a.err, kErrBadIndex);
         // 128 consecutive keys (a near-dense selection): two tiled copies
         const int last = __shfl_sync(0xffffffffu, j[3], 31);
+        // (every lane's four keys exactly the next ones: a list entry out of
+        // order or repeated keeps the gather path)
         const bool contiguous = td.valid == 128 && last - first == 127 && first >= 0 &&
-                                last < a.g.L;
+                                last < a.g.L &&
+                                __all_sync(0xffffffffu, j[0] == first + 4 * lane &&
+                                                            j[1] == first + 4 * lane + 1 &&
+                                                            j[2] == first + 4 * lane + 2 &&
+                                                            j[3] == first + 4 * lane + 3);
         if (lane == 0) mbar_arrive_expect_tx(kf, kTileBytes);
         __syncwarp();
         if (contiguous) {

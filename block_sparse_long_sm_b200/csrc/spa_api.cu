@@ -247,17 +247,43 @@ __device__ __align__(256) uint8_t g_static_scratch[kStaticScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_static_mutex;
 void* g_static_ptr[kMaxDevices] = {};
+void* g_static_ctx[kMaxDevices] = {};
 
-// Device address of g_static_scratch on the current device, looked up once
-// per device (the host-side name is only a stand-in, not a device address).
+typedef int (*CtxGetCurrentFn)(void**);
+
+// The current context of the calling thread (driver API through the runtime's
+// entry-point lookup, so the library needs no link against libcuda).
+void* current_context() {
+  static CtxGetCurrentFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return nullptr;
+    fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  }
+  void* ctx = nullptr;
+  return fn(&ctx) == 0 ? ctx : nullptr;
+}
+
+// Device address of g_static_scratch on the current device (the host-side
+// name is only a stand-in, not a device address).  Looked up with the device
+// current on the first call of each device, and again whenever the device's
+// context has changed since (after a cudaDeviceReset the old address is gone).
 void* static_scratch_ptr() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  // makes the device's primary context current (no allocation)
+  if (cudaSetDevice(dev) != cudaSuccess) return nullptr;
+  void* ctx = current_context();
+  if (!ctx) return nullptr;
   std::lock_guard<std::mutex> lock(g_static_mutex);
-  if (!g_static_ptr[dev]) {
+  if (!g_static_ptr[dev] || g_static_ctx[dev] != ctx) {
     void* ptr = nullptr;
     if (cudaGetSymbolAddress(&ptr, g_static_scratch) != cudaSuccess) return nullptr;
     g_static_ptr[dev] = ptr;
+    g_static_ctx[dev] = ctx;
   }
   return g_static_ptr[dev];
 }
@@ -297,7 +323,12 @@ SPA_API spa_status sparse_prefill_plan_static(const spa_params* p, const void* q
   const StaticLayout sl = static_layout(p, lo);
   if (sl.total > kStaticScratchBytes) return SPA_ERR_UNSUPPORTED;
   const int B = p->batch, Hq = p->heads_q, Hkv = p->heads_kv, L = p->seq_len;
-  if (B == 0 || L == 0) return SPA_OK;
+  if (B == 0 || L == 0) {
+    // nothing to select; the caller's error word still reports this call
+    if (error_word && cudaMemsetAsync(error_word, 0, sizeof(uint32_t), stream) != cudaSuccess)
+      return SPA_ERR_CUDA;
+    return SPA_OK;
+  }
   if (!q || !k || !counts || !aligned16(q) || !aligned16(k) ||
       (reinterpret_cast<uintptr_t>(counts) & 3u))
     return SPA_ERR_INVALID;

@@ -205,7 +205,10 @@ SPA_API spa_status sparse_prefill_stats(const spa_params* p, const void* workspa
  *
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture.  All calls share the array and it keeps the last
+ * before any stream capture.  A call that finds the device's context changed
+ * since (after cudaDeviceReset) looks the address up again, so it too should
+ * come before any capture.  For an empty problem (B or L zero) nothing is
+ * launched and *error_word, when given, is set to zero.  All calls share the array and it keeps the last
  * call's contents (the header is cleared on every call); calls that overlap
  * on the GPU -- on different streams or from different threads -- race and
  * must be serialised by the caller. */

@@ -43,11 +43,12 @@ def _static_plan(p, q, k, n_lists):
     return counts, lists[:n_lists], int(err.item())
 
 
-def _case(w, L, theta, sink, local):
+def _case(w, L, theta, sink, local, step=1):
     inp = generate(w.with_(sink=sink, local=local), seq_len=L)
     q, k = to_dev(inp.q), to_dev(inp.k)
     B, Hq, Hkv = w.batch, w.heads_q, w.heads_kv
-    p = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=sink, local=local, theta=theta)
+    p = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=sink, local=local, theta=theta,
+                        step=step)
     return p, q, k
 
 
@@ -80,6 +81,28 @@ def test_static_plan_matches_workspace_plan_on_back_to_back_calls():
     kept2 = _check_same(p2, q2, k2)
     assert _check_same(p1, q1, k1) == kept1
     assert kept1 > 0 and kept2 > 0
+
+
+@pytest.mark.parametrize("step", [2, 3])
+def test_static_plan_matches_workspace_plan_with_grouped_query_blocks(step):
+    # the workspace plan unions a group of query blocks inside its fused
+    # selection kernel when step is a power of two (step 2) and through the
+    # separate compaction otherwise (step 3); the static plan always takes
+    # the compaction path, over scratch the previous call left behind
+    p, q, k = _case(C1_LLAMA_32K, 2500, 3.0, 128, 256, step=step)
+    kept = _check_same(p, q, k)
+    p1, q1, k1 = _case(C0_TINY, 4096, 2.5, 64, 128, step=step)
+    assert _check_same(p1, q1, k1) > 0
+    assert _check_same(p, q, k) == kept > 0
+
+
+def test_static_plan_empty_problem_clears_the_error_word():
+    p = spa.make_params(0, 4, 2, 1024, mode="anchor", sink=64, local=128, theta=3.0)
+    dummy = torch.empty(16, dtype=torch.int32, device="cuda")
+    err = torch.full((1,), 7, dtype=torch.int32, device="cuda")
+    assert sparse_prefill_plan_static(p, dummy, dummy, dummy, dummy, 0, err) == spa.SPA_OK
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
 
 
 def test_static_plan_rejects_problems_beyond_its_scratch():
