@@ -205,15 +205,16 @@ def run_reference(args, w: Workload):
     print(json.dumps(line), flush=True)
 
 
-def _config(w: Workload, args):
-    return {"workload": w.name, "attn_variant": "window_tiles" if getattr(args, "window_tiles", False)
-            else "gather_tiles", "batch": w.batch, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
+def _config(w: Workload, args, world: int = 1):
+    return {"workload": w.name, "batch": w.batch, "heads_q": w.heads_q, "heads_kv": w.heads_kv,
             "seq_len": w.seq_len, "head_dim": 128, "causal": True, "mode": args.mode,
             "theta": args.theta, "sink": w.sink, "local": w.local, "block_q": 128,
             "l2": f"inputs ({2 * 128 * w.seq_len * w.batch * (w.heads_q + 2 * w.heads_kv) / 1e9:.2f} GB) "
                   + ("larger than L2 (126 MB); no flush" if w.seq_len * w.batch * (w.heads_q + 2 * w.heads_kv) * 256 > 126e6
                      else "smaller than L2"),
-            "parallelism": "independent layer per GPU"}
+            "parallelism": (f"one layer split by kv head over {world} GPUs"
+                            if getattr(args, "split", False) and world > 1
+                            else "independent layer per GPU")}
 
 
 def main():
@@ -235,15 +236,15 @@ def main():
     ap.add_argument("--fp8", action="store_true",
                     help="E4M3 quantisation + FP8 attention over the plan instead of the "
                          "headline step")
-    ap.add_argument("--window-tiles", action="store_true",
-                    help="paired attention with contiguous masked windows for near-dense "
-                         "selected keys (SPA_DEBUG_WINDOW_TILES)")
+    ap.add_argument("--split", action="store_true",
+                    help="under torchrun, split one layer by kv head across the ranks (strong "
+                         "scaling) instead of running one layer per rank (weak scaling)")
     ap.add_argument("--key-mass", action="store_true",
                     help="key mass from the prefill LSE over the plan instead of the headline step")
     args = ap.parse_args()
     w = CONFIGS[args.config]
     if args.sweep:
-        sweep(window_tiles=args.window_tiles)
+        sweep()
         return
     if args.decode:
         decode_bench(args, w)
@@ -279,13 +280,21 @@ def main():
     B, Hq, Hkv, L = w.batch, w.heads_q, w.heads_kv, w.seq_len
     o = torch.empty((B, Hq, L, 128), dtype=torch.bfloat16, device=dev)
     p = spa.make_params(B, Hq, Hkv, L, mode=args.mode, sink=w.sink, local=w.local,
-                        theta=args.theta, tau=w.tau, block_k=w.block_k if args.mode == "sale" else None,
-                        debug_flags=(spa.SPA_DEBUG_WINDOW_TILES if args.window_tiles else 0))
+                        theta=args.theta, tau=w.tau, block_k=w.block_k if args.mode == "sale" else None)
+    # --split: this rank's kv heads of the one layer (all of it on one GPU)
+    split = args.split and world > 1
+    if split:
+        from block_sparse_long_sm_b200.shard import rank_sub_layer
+        sub = rank_sub_layer(p, world, rank)
+        p = sub.params
+        qa, ka, va, oa, _ = sub.pointers(q, k, v, o)
+    else:
+        qa, ka, va, oa = q, k, v, o
     ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
 
     def step():
-        spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream), "plan")
-        spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None, stream=stream), "attn")
+        spa.check(spa.sparse_prefill_plan(p, qa, ka, ws, stream=stream), "plan")
+        spa.check(spa.sparse_prefill_attn(p, qa, ka, va, ws, oa, None, stream=stream), "attn")
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -304,9 +313,9 @@ def main():
         t_start.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
-            spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream), "plan")
+            spa.check(spa.sparse_prefill_plan(p, qa, ka, ws, stream=stream), "plan")
             ev[i][1].record(stream)
-            spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None, stream=stream), "attn")
+            spa.check(spa.sparse_prefill_attn(p, qa, ka, va, ws, oa, None, stream=stream), "attn")
             ev[i][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -320,7 +329,13 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
     ms_step = total_ms / args.steps
-    value = flops_step * world * args.steps / (total_ms / 1e3) / 1e12
+    layer_flops = flops_step * world            # weak: every rank runs a whole layer
+    if split:
+        # strong: the ranks' kept FLOPs add up to the one layer's
+        t = torch.tensor([float(flops_step)], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        layer_flops = float(t.item())
+    value = layer_flops * args.steps / (total_ms / 1e3) / 1e12
     peaks = _peaks()
     attn_avg = sum(attn_ms) / len(attn_ms)
     achieved = flops_step / (attn_avg / 1e3) / 1e12
@@ -336,8 +351,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms_step, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": _config(w, args),
+            "scaling": "strong" if split else "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": _config(w, args, world),
             "plan_ms": statistics.median(plan_ms), "attn_ms": statistics.median(attn_ms),
             "kept_fraction": stats.kept_pairs / stats.dense_pairs,
             "kept_flops_per_layer": flops_step,
@@ -360,7 +375,7 @@ def main():
         dist.destroy_process_group()
 
 
-def sweep(window_tiles: bool = False):
+def sweep():
     """Kept fraction vs time and vs tensor peak over theta (the density sweep
     of the 128K Llama layer, its B = 4, L = 16384 variant and the 64K Qwen
     layer with half its kv heads diffuse).  One JSON line per point; theta =
@@ -406,8 +421,7 @@ def sweep(window_tiles: bool = False):
         del wsd
         for theta in thetas:
             p = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=w.sink, local=w.local,
-                                theta=theta,
-                                debug_flags=spa.SPA_DEBUG_WINDOW_TILES if window_tiles else 0)
+                                theta=theta)
             ws = torch.empty(spa.sparse_prefill_workspace_bytes(p), dtype=torch.uint8, device=dev)
             plan_ms = timed(lambda: spa.check(spa.sparse_prefill_plan(p, q, k, ws, stream=stream)))
             attn_ms = timed(lambda: spa.check(spa.sparse_prefill_attn(p, q, k, v, ws, o, None,
@@ -418,7 +432,6 @@ def sweep(window_tiles: bool = False):
             alg_bytes = 2 * B * Hq * L * 128 + 2 * B * Hkv * L * 128 + 4 * s.kept_candidates
             print(json.dumps({
                 "sweep": "density", "workload": w.name, "theta": theta,
-                "attn_variant": "window_tiles" if window_tiles else "gather_tiles",
                 "kept_fraction": s.kept_pairs / s.dense_pairs,
                 "kept_candidates_fraction": s.kept_candidates / max(1, s.candidates),
                 "plan_ms": plan_ms, "attn_ms": attn_ms, "step_ms": plan_ms + attn_ms,
@@ -802,8 +815,7 @@ def bench_extras(spa, torch, w, args, q, k, v, o, q_h, k_h, v_h, stream, dev, st
     # besides the headline's value, and SALE at a tau that skips key blocks
     points = []
     for theta in (3.0, 7.0):
-        pt = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=w.sink, local=w.local, theta=theta,
-                             debug_flags=spa.SPA_DEBUG_WINDOW_TILES if args.window_tiles else 0)
+        pt = spa.make_params(B, Hq, Hkv, L, mode="anchor", sink=w.sink, local=w.local, theta=theta)
         wst = torch.empty(spa.sparse_prefill_workspace_bytes(pt), dtype=torch.uint8, device=dev)
         points.append(_operating_point(spa, torch, timed, pt, wst, q, k, v, o, stream, peaks,
                                        dense_ms, dict(mode="anchor", theta=theta)))

@@ -11,7 +11,7 @@ ImportError (there is no fallback).
 import importlib
 
 _BINDING_NAMES = (
-    "EXPORTED", "LIB_PATH", "MODES", "SPA_DEBUG_STALL_ATTN", "SPA_DEBUG_WINDOW_TILES",
+    "EXPORTED", "LIB_PATH", "MODES", "SPA_DEBUG_STALL_ATTN",
     "SPA_ERR_CUDA", "SPA_ERR_INVALID", "SPA_ERR_TIMEOUT", "SPA_ERR_UNSUPPORTED",
     "SPA_ERR_WORKSPACE", "SPA_MODE_ANCHOR", "SPA_MODE_DENSE", "SPA_MODE_SALE", "SPA_OK",
     "SpaError", "SpaParams", "SpaStats", "check", "kept_flops", "make_params",

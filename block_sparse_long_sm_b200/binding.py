@@ -21,7 +21,6 @@ LIB_PATH = os.path.join(_PKG, "lib", "libspa.so")
 SPA_OK, SPA_ERR_INVALID, SPA_ERR_UNSUPPORTED, SPA_ERR_WORKSPACE, SPA_ERR_CUDA, SPA_ERR_TIMEOUT = range(6)
 SPA_MODE_ANCHOR, SPA_MODE_SALE, SPA_MODE_DENSE = 0, 1, 2
 SPA_DEBUG_STALL_ATTN = 0x1
-SPA_DEBUG_WINDOW_TILES = 0x2
 MODES = {"anchor": SPA_MODE_ANCHOR, "sale": SPA_MODE_SALE, "dense": SPA_MODE_DENSE}
 
 EXPORTED = ("sparse_prefill_workspace_bytes", "sparse_prefill_plan", "sparse_prefill_attn",

@@ -41,28 +41,6 @@ constexpr uint32_t kAttnSmemBytes =
     1024u + kTileBytes + kAttnStages * 2u * kTileBytes + 256u;
 static_assert(kAttnSmemBytes <= 232448u, "more shared memory than a CTA may use");
 
-// 2^f on [-1/2, 1/2], degree 3, minimax in relative error (max 7.5e-5); the
-// fit is reproduced by csrc/exp2_poly_fit.py.
-constexpr float kExp2C0 = 0.999928117f;
-constexpr float kExp2C1 = 0.693260968f;
-constexpr float kExp2C2 = 0.242610544f;
-constexpr float kExp2C3 = 0.0551713221f;
-
-// 2^x on the FMA pipe (Cody-Waite range reduction): x = n + f with
-// n = round(x) added to the exponent field and f in [-1/2, 1/2] through the
-// polynomial.  x is clamped at -126, so masked (-inf) entries give
-// 2^-126 ~ 1e-38, which vanishes in every sum.
-__device__ __forceinline__ float poly_exp2(float x) {
-  x = fmaxf(x, -126.0f);
-  const float t = x + 12582912.0f;                       // 1.5 * 2^23: round to integer
-  const float n = t - 12582912.0f;
-  const float f = x - n;
-  float p = fmaf(kExp2C3, f, kExp2C2);
-  p = fmaf(p, f, kExp2C1);
-  p = fmaf(p, f, kExp2C0);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 struct AttnArgs {
   int B, Hq, Hkv, L, nqb, group;
   int sink, local;
@@ -73,10 +51,13 @@ struct AttnArgs {
   long long list_per_head;    // list elements per (b, h)
   long long cap_a;            // local + sink (capacity prefix constant), in keys
   int list_unit;              // 1 (keys) or bk (SALE: list holds key-block ids)
-  const int* pair_counts;     // paired kernel: union entries per (b, head pair, qb)
-  const uint32_t* pair_lists; // paired kernel: tagged union lists
-  const int* pair_split;      // paired kernel: union entries shared with head A's list
-  long long pair_per_head;    // list elements per (b, head pair)
+  const uint4* tmask;         // paired kernel: candidate-tile masks [B*Hq][tmask_per_head]
+  long long tmask_per_head;
+  int tc;                     // tmask_c(sink, local)
+  const uint32_t* tbits;      // paired kernel: tile bitmaps [B*Hq*nqb][3][tbit_words]
+  int tbit_words;
+  const __nv_bfloat16* k;     // paired kernel: K and V rows for the gathered tiles
+  const __nv_bfloat16* v;
   __nv_bfloat16* o;
   float* lse;
   uint32_t* err;

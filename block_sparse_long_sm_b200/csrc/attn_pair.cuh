@@ -3,26 +3,44 @@
 //
 // Same computation as sparse_attn_kernel (AnchorAttention Sec. 3.4 /
 // SALE Computation Pass, FlashAttention online softmax), organised so that
-// the exponentials of one head overlap the tensor-core work of the other:
+// the exponentials of one head overlap the tensor-core work of the other.
 //
-//   * one CTA = (b, kv head, query block, head pair (2p, 2p+1)); the key
-//     sequence is sink tiles, the tiles of the pair's *union* list (every
-//     entry carries which of the two heads kept it; up to the first entry
-//     where the heads differ the union is head A's own list), and local
-//     tiles;
-//   * warp 8 loads Q of both heads once and K/V tiles into rings of 3 (K) and
-//     2 (V) stages, gathering selected rows with TMA gather4, and publishes a
-//     128-bit membership mask per head for each selected tile;
-//   * warp 9 issues tcgen05.mma in the order PV_A(t), QK_A(t+1), PV_B(t),
-//     QK_B(t+1): the tensor core runs one head's GEMMs while the other head's
-//     softmax works.  P is written by the softmax into the first 64 columns of
-//     its own S accumulator and read from there by the PV GEMM; the next QK
-//     GEMM into the same columns is issued after that PV GEMM, and tcgen05
-//     MMAs from one thread execute in issue order;
-//   * warps 0-3 are head A's softmax and warps 4-7 head B's (thread = row =
-//     TMEM lane).  Per tile: row max, then
-//     exponentials + P: S is read once into registers (four TMEM loads, one
-//     wait); P overwrites S's first 64 columns.
+// One CTA = (b, kv head, query block, head pair (2p, 2p+1)).  Its key tiles:
+//   sink tiles       keys [0, sink_end), contiguous;
+//   dense tiles      candidate tiles (128 aligned keys) in which the two
+//                    heads keep at least kTileDenseMin keys together: loaded
+//                    contiguously, the keys a head did not keep masked out of
+//                    its softmax;
+//   gathered tiles   the kept keys of the sparser candidate tiles, 128 at a
+//                    time (the last one padded), copied row by row;
+//   local tiles      keys [ls, row0 + 128), contiguous; the last one is the
+//                    causally masked diagonal.
+// The candidate tiles come from the plan's tile masks (one 128-bit keep mask
+// per head, query block and candidate tile), so the kernel reads 32 bytes of
+// selection per 128 candidate keys and no index list.  Attention over a key
+// set does not depend on the order of its tiles.
+//
+// Roles (384 threads, 3 warpgroups; warps 10 and 11 have no role):
+//   warp 8       producer: Q of both heads once; per tile it picks the keys
+//                (sink, dense, gathered or local), publishes a descriptor and
+//                the two heads' column masks through the tile's tag barrier,
+//                and loads the tile with TMA into rings of 3 (K) and 2 (V)
+//                stages: contiguous tiles as two 64-column boxes per operand.
+//                Gathered tiles are copied row by row with TMA gather4 (four
+//                rows per instruction, issued by the 32 lanes);
+//   warp 9       TMEM allocation and the single MMA-issuing thread, in the
+//                order PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1), so the tensor
+//                core works on one head while the other head's softmax runs.
+//                P is written by the softmax into the first 64 columns of its
+//                own S accumulator and read there by the PV GEMM; the next QK
+//                GEMM into the same columns is issued after that PV GEMM
+//                (tcgen05 MMAs of one thread execute in issue order);
+//   warps 0-3 / 4-7  softmax of head A / B, thread = query row = TMEM lane.
+//
+// The number of tiles depends on the masks, so every tile carries a
+// descriptor (valid columns, causal, masked, last, gathered); the MMA and
+// softmax warps stop after the tile marked last (a local tile: there is
+// always at least one, the diagonal).
 //
 // TMEM columns: S_A [0,128) (P_A in [0,64)), S_B [128,256) (P_B in
 // [128,192)), O_A [256,384), O_B [384,512).
@@ -31,21 +49,21 @@
 #include "attn.cuh"
 #include "ptx.cuh"
 
-// One exponential pair in SPA_EXP2_POLY_EVERY goes through the FMA-pipe
-// polynomial instead of MUFU (0: none).
-#ifndef SPA_EXP2_POLY_EVERY
-#define SPA_EXP2_POLY_EVERY 0
-#endif
-
 namespace spa {
 
 constexpr int kPairKStages = 3;
 constexpr int kPairVStages = 2;
 constexpr int kPairThreads = 384;   // 3 warpgroups: softmax A, softmax B, load + MMA
-constexpr uint32_t kPairBarBytes = 1024u;
+constexpr uint32_t kPairBarBytes = 1024u;   // barriers, masks, descriptors, staged keys
 constexpr uint32_t kPairSmemBytes =
     1024u + 2u * kTileBytes + (kPairKStages + kPairVStages) * kTileBytes + kPairBarBytes;
 static_assert(kPairSmemBytes <= 232448u, "more shared memory than a CTA may use");
+
+// tile descriptor bits (bits 0-8: valid columns)
+constexpr uint32_t kDescCausal = 1u << 9;
+constexpr uint32_t kDescMasked = 1u << 10;
+constexpr uint32_t kDescLast = 1u << 11;
+constexpr uint32_t kDescGather = 1u << 12;
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
@@ -73,10 +91,12 @@ __device__ __forceinline__ void tmem_st32_halves(uint32_t taddr, const uint32_t*
 }
 
 struct PairItem {
-  AttnItem it;     // geometry; it.h is head A, it.n_sel counts union keys
-  int pair;        // b * Hq / 2 + hA / 2
-  int split;       // union entries before the two heads' lists first differ
-  long long a_off; // head A's list of this block: the union's first `split` entries
+  AttnItem it;          // geometry; it.h is head A
+  int n_ct;             // candidate tiles of the block
+  const uint4* ma;      // head A's tile masks of this block
+  const uint4* mb;      // head B's
+  const uint32_t* ba;   // head A's tile bitmaps of this block (non-empty, dense, full)
+  const uint32_t* bb;   // head B's
 };
 
 __device__ __forceinline__ PairItem pair_item(const AttnArgs& a, int x) {
@@ -91,48 +111,33 @@ __device__ __forceinline__ PairItem pair_item(const AttnArgs& a, int x) {
   it.b = bkv / a.Hkv;
   it.kvh = bkv - it.b * a.Hkv;
   it.h = it.kvh * a.group + 2 * pp;
-  pi.pair = it.b * (a.Hq / 2) + it.h / 2;
   it.row0 = it.qb * 128;
   it.le = min(it.row0 + 128, a.L);
   it.ls = max(0, it.row0 + 128 - a.local);
   it.sink_end = min(a.sink, it.ls);
-  pi.split = 0;
-  pi.a_off = 0;
+  it.n_sel = 0;
+  it.n_sel_t = 0;
+  it.list_off = 0;
+  pi.n_ct = 0;
+  pi.ma = nullptr;
+  pi.mb = nullptr;
+  pi.ba = nullptr;
+  pi.bb = nullptr;
   if (a.mode == kModeDense) {
     it.n_sink_t = 0;
-    it.n_sel = 0;
     it.loc_start = 0;
-    it.list_off = 0;
   } else {
     it.n_sink_t = (it.sink_end + 127) / 128;
-    const int cnt = a.pair_counts[(long long)pi.pair * a.nqb + it.qb];
-    it.n_sel = cnt * a.list_unit;
     it.loc_start = it.ls;
-    it.list_off = (long long)pi.pair * a.pair_per_head +
-                  cap_prefix(it.qb, 128, a.cap_a) / a.list_unit;
-    pi.split = a.pair_split[(long long)pi.pair * a.nqb + it.qb];
-    pi.a_off = ((long long)it.b * a.Hq + it.h) * a.list_per_head +
-               cap_prefix(it.qb, 128, a.cap_a) / a.list_unit;
+    pi.n_ct = tmask_tiles(it.qb, a.tc);
+    const long long bhA = (long long)it.b * a.Hq + it.h;
+    pi.ma = a.tmask + bhA * a.tmask_per_head + tmask_prefix(it.qb, a.tc);
+    pi.mb = pi.ma + a.tmask_per_head;
+    pi.ba = a.tbits + (bhA * a.nqb + it.qb) * 3 * a.tbit_words;
+    pi.bb = pi.ba + (long long)a.nqb * 3 * a.tbit_words;
   }
-  it.n_sel_t = (it.n_sel + 127) / 128;
   it.n_loc_t = (it.le - it.loc_start + 127) / 128;
   return pi;
-}
-
-// Union entry of selected ordinal n: key index and 2-bit membership tag.
-// While the two heads' lists agree, the union is head A's list (both heads
-// keep every entry); the plan writes union entries only from the first
-// difference on.
-__device__ __forceinline__ void pair_sel(const AttnArgs& a, const PairItem& pi, int n, int& key,
-                                         uint32_t& tag) {
-  const int ne = n / a.list_unit;
-  const bool shared = ne < pi.split;
-  const uint32_t* src = shared ? reinterpret_cast<const uint32_t*>(a.lists) + pi.a_off
-                               : a.pair_lists + pi.it.list_off;
-  const uint32_t e = src[ne] | (shared ? (3u << 30) : 0u);
-  tag = e >> 30;
-  const int idx = static_cast<int>(e & 0x3FFFFFFFu);
-  key = a.list_unit == 1 ? idx : idx * a.list_unit + n % a.list_unit;
 }
 
 __global__ void __launch_bounds__(kPairThreads, 1)
@@ -162,8 +167,16 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   const uint32_t bar_stall = bar_sfull0 + 48u;
   const uint32_t bar_tag0 = bar_sfull0 + 56u;                                         // [vstages]
   uint32_t* tags = reinterpret_cast<uint32_t*>(bar_area + 256);   // [vstage][head][4 words]
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 512);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 320);
   volatile uint32_t* abort_flag = tmem_holder + 1;
+  // per V slot, the descriptor of the tile in it: valid columns (bits 0-8)
+  // and the kDesc* flags; written by the producer before it arrives on the
+  // slot's tag barrier
+  uint32_t* tdesc = reinterpret_cast<uint32_t*>(bar_area + 336);
+  // the next gathered tile's keys, row by row (index | head A kept it << 30 |
+  // head B kept it << 31), while the producer collects them; padding rows
+  // repeat row 0's key with neither head's bit
+  uint32_t* stage = reinterpret_cast<uint32_t*>(bar_area + 512);   // [128]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -208,18 +221,14 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 
   const PairItem pi = pair_item(a, blockIdx.x);
   const AttnItem& it = pi.it;
-  const int T = it.n_sink_t + it.n_sel_t + it.n_loc_t;
   const int kv_row0 = (it.b * a.Hkv + it.kvh) * a.L;
 
-  // Register split: the load/MMA warpgroup needs few registers, the softmax
-  // warpgroups hold a full 128-column S row each.  Launched with 168 per
-  // thread (384 threads): 128 x (168 - 40) = 256 x (232 - 168).
-  if (warp >= 8) {
   // Register split: the load/MMA warpgroup (warps 8-11, executing this one
   // instruction together) needs few registers, the softmax warpgroups hold a
   // full 128-column S row each.  Launched with 168 per thread (384 threads):
-  // 128 x 80 + 256 x 208 <= 384 x 168.
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
+  // 128 x 88 + 256 x 208 = 384 x 168.
+  if (warp >= 8) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
   if (warp == 8) {
     // ------------------------------------------------------------- producer
     int issued = 0;
@@ -231,32 +240,219 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       tma_load_2d(s_q + kTileBytes, &tm_q, bar_q, 0, qrow + a.L);
       tma_load_2d(s_q + kTileBytes + kHalfBytes, &tm_q, bar_q, 64, qrow + a.L);
     }
-    // Union entries of this lane's four rows of a selected tile, fetched one
-    // tile ahead (padding rows repeat the first key with an empty tag).
-    auto fetch = [&](int t, int (&j)[4], uint32_t (&tg)[4]) {
-      const TileDesc td = tile_desc(it, t);
-      if (!td.gather) return;
-      int first;
-      uint32_t ftag;
-      pair_sel(a, pi, td.key0, first, ftag);
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int row = lane * 4 + r;
-        if (row < td.valid) {
-          pair_sel(a, pi, td.key0 + row, j[r], tg[r]);
-        } else {
-          j[r] = first;
-          tg[r] = 0u;
-        }
+    const int kt0 = a.sink / 128;
+    const int W = a.tbit_words;
+    const int nw = (pi.n_ct + 31) / 32;            // bitmap words of this block
+    // The bitmaps are read 32 words (1024 tiles) at a time, lane l holding
+    // word l of the chunk.
+    // Dense tiles: set in either head's dense bitmap; full when both heads
+    // keep all 128 keys.
+    int dchunk = 0, dwi = -1;
+    uint32_t dword = 0u, fword = 0u;               // this lane's word of the chunk
+    uint32_t dbits = 0u, fbits = 0u;               // the word in use: tiles left, full tiles
+    auto load_dense_chunk = [&](int c) {
+      const int wi = 32 * c + lane;
+      dword = fword = 0u;
+      if (wi < nw) {
+        dword = pi.ba[W + wi] | pi.bb[W + wi];
+        fword = pi.ba[2 * W + wi] & pi.bb[2 * W + wi];
       }
     };
-    int nj[4] = {0, 0, 0, 0};
-    uint32_t ntg[4] = {0u, 0u, 0u, 0u};
-    if (T > 0) fetch(0, nj, ntg);
-    for (int t = 0; t < T; ++t) {
-      int j[4] = {nj[0], nj[1], nj[2], nj[3]};
-      const uint32_t tg[4] = {ntg[0], ntg[1], ntg[2], ntg[3]};
-      if (t + 1 < T) fetch(t + 1, nj, ntg);
+    // next dense tile (candidate index) and whether it is full, or -1
+    auto next_dense = [&](bool& full) -> int {
+      while (dbits == 0u) {
+        if (32 * dchunk >= nw) return -1;
+        const uint32_t cand = __ballot_sync(0xffffffffu, dword != 0u) &
+                              (dwi < 31 ? (0xffffffffu << (dwi + 1)) : 0u);
+        if (cand) {
+          dwi = __ffs(cand) - 1;
+          dbits = __shfl_sync(0xffffffffu, dword, dwi);
+          fbits = __shfl_sync(0xffffffffu, fword, dwi);
+        } else {
+          ++dchunk;
+          dwi = -1;
+          if (32 * dchunk < nw) load_dense_chunk(dchunk);
+        }
+      }
+      const int b = __ffs(dbits) - 1;
+      dbits &= dbits - 1u;
+      full = ((fbits >> b) & 1u) != 0u;
+      return 32 * (32 * dchunk + dwi) + b;
+    };
+    // Gathered tiles: the keys of the tiles that are non-empty and not dense,
+    // taken a window at a time (the sparse tiles of one bitmap word, lane j
+    // holding the j-th), the next window's masks loaded ahead.
+    int sc = 0, swi = -1;
+    bool s_done = nw == 0;
+    uint32_t sword = 0u;                           // this lane's sparse word of chunk sc
+    auto load_sparse_chunk = [&](int c) {
+      const int wi = 32 * c + lane;
+      sword = 0u;
+      if (wi < nw) sword = (pi.ba[wi] | pi.bb[wi]) & ~(pi.ba[W + wi] | pi.bb[W + wi]);
+    };
+    bool p_valid = false;                          // prefetched window
+    int p_n = 0, p_tile = 0;
+    uint4 p_a = make_uint4(0u, 0u, 0u, 0u), p_b = p_a;
+    auto scan_next = [&]() {
+      p_valid = false;
+      while (!s_done) {
+        const uint32_t cand = __ballot_sync(0xffffffffu, sword != 0u) &
+                              (swi < 31 ? (0xffffffffu << (swi + 1)) : 0u);
+        if (cand) {
+          swi = __ffs(cand) - 1;
+          const uint32_t word = __shfl_sync(0xffffffffu, sword, swi);
+          p_n = __popc(word);
+          if (lane < p_n) {
+            p_tile = 32 * (32 * sc + swi) + static_cast<int>(__fns(word, 0, lane + 1));
+            p_a = pi.ma[p_tile];
+            p_b = pi.mb[p_tile];
+          }
+          p_valid = true;
+          return;
+        }
+        ++sc;
+        swi = -1;
+        if (32 * sc >= nw) {
+          s_done = true;
+          return;
+        }
+        load_sparse_chunk(sc);
+      }
+    };
+    bool g_valid = false;                          // window in use
+    int g_tile = 0, g_cnt = 0;
+    uint4 g_a = p_a, g_b = p_a;
+    int j0 = 0, cons = 0;                          // first lane not used up, its keys taken
+    auto take_window = [&]() {
+      g_valid = p_valid;
+      if (!g_valid) return;
+      g_tile = p_tile;
+      g_a = p_a;
+      g_b = p_b;
+      g_cnt = lane < p_n ? __popc(g_a.x | g_b.x) + __popc(g_a.y | g_b.y) +
+                               __popc(g_a.z | g_b.z) + __popc(g_a.w | g_b.w)
+                         : 0;
+      j0 = 0;
+      cons = 0;
+      scan_next();
+    };
+    if (nw > 0) {
+      load_dense_chunk(0);
+      load_sparse_chunk(0);
+      scan_next();
+      take_window();
+    }
+    int phase = 0;        // 0 sink, 1 dense, 2 gathered, 3 local tiles
+    int n_sink = 0, n_loc = 0;
+    // The next tile, prepared while the previous tile's loads are in flight:
+    // its descriptor, its first key (contiguous tiles), lane l's four rows
+    // 4 l .. 4 l + 3 (gathered tiles) and, in lanes 0-7, word l of the two
+    // heads' column masks (0-3 head A, 4-7 head B).
+    uint32_t nx_desc = 0u;
+    int nx_key0 = 0;
+    int nx_row[4] = {0, 0, 0, 0};
+    uint32_t nx_mask = 0u;
+    auto prepare = [&]() {
+      nx_desc = 0u;
+      if (phase == 0) {
+        if (n_sink < it.n_sink_t) {
+          nx_key0 = 128 * n_sink++;
+          nx_desc = static_cast<uint32_t>(min(128, it.sink_end - nx_key0));
+          return;
+        }
+        phase = 1;
+      }
+      if (phase == 1) {
+        bool full = false;
+        const int j = nw > 0 ? next_dense(full) : -1;
+        if (j >= 0) {
+          if (!full && lane < 8)
+            nx_mask = reinterpret_cast<const uint32_t*>(lane < 4 ? pi.ma + j : pi.mb + j)[lane & 3];
+          nx_key0 = 128 * (kt0 + j);
+          nx_desc = 128u | (full ? 0u : kDescMasked);
+          return;
+        }
+        phase = 2;
+      }
+      if (phase == 2) {
+        // the next 128 keys of the sparse tiles
+        int filled = 0;
+        while (filled < 128 && g_valid) {
+          const int skip = lane == j0 ? cons : 0;
+          const int cnt = lane >= j0 ? g_cnt - skip : 0;
+          int incl = cnt;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+          }
+          const int excl = incl - cnt;
+          const int tot = __shfl_sync(0xffffffffu, incl, 31);
+          const int take = min(tot, 128 - filled);
+          if (cnt > 0 && excl < take) {
+            // this lane's tile: its keys of rank skip, skip + 1, ... go to
+            // slots filled + excl, ... while they are below filled + take
+            const uint32_t ua[4] = {g_a.x, g_a.y, g_a.z, g_a.w};
+            const uint32_t ub[4] = {g_b.x, g_b.y, g_b.z, g_b.w};
+            const int base_key = 128 * (kt0 + g_tile);
+            int r = 0;
+            for (int w = 0; w < 4; ++w) {
+              uint32_t rem = ua[w] | ub[w];
+              while (rem) {
+                const int bpos = __ffs(rem) - 1;
+                rem &= rem - 1u;
+                if (r >= skip) {
+                  const int pos = excl + r - skip;
+                  if (pos < take)
+                    stage[filled + pos] = static_cast<uint32_t>(base_key + 32 * w + bpos) |
+                                          (((ua[w] >> bpos) & 1u) << 30) |
+                                          (((ub[w] >> bpos) & 1u) << 31);
+                }
+                ++r;
+              }
+            }
+          }
+          filled += take;
+          if (take == tot) {
+            take_window();
+          } else {
+            // the window continues at the lane holding the first key not taken
+            const uint32_t cut = __ballot_sync(0xffffffffu, cnt > 0 && excl <= take && take < excl + cnt);
+            const int J = __ffs(cut) - 1;
+            const int eJ = __shfl_sync(0xffffffffu, excl, J);
+            cons = (J == j0 ? cons : 0) + (take - eJ);
+            j0 = J;
+          }
+        }
+        __syncwarp();
+        if (filled > 0) {
+          const uint32_t first = stage[0] & 0x3FFFFFFFu;
+          for (int r = filled + lane; r < 128; r += 32) stage[r] = first;
+          __syncwarp();
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            nx_row[r] = kv_row0 + static_cast<int>(stage[4 * lane + r] & 0x3FFFFFFFu);
+          // column masks: row 32 w + l of the tile is bit l of word w
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const uint32_t e = stage[32 * w + lane];
+            const uint32_t ma = __ballot_sync(0xffffffffu, (e >> 30) & 1u);
+            const uint32_t mb = __ballot_sync(0xffffffffu, (e >> 31) & 1u);
+            if (lane == w) nx_mask = ma;
+            if (lane == 4 + w) nx_mask = mb;
+          }
+          __syncwarp();   // the staging buffer may be refilled for the tile after
+          nx_desc = 128u | kDescMasked | kDescGather;
+          return;
+        }
+        phase = 3;
+      }
+      nx_key0 = it.loc_start + 128 * n_loc++;
+      nx_desc = static_cast<uint32_t>(min(128, it.le - nx_key0)) |
+                (nx_key0 == it.row0 ? kDescCausal : 0u) | (n_loc == it.n_loc_t ? kDescLast : 0u);
+    };
+    prepare();
+    for (int t = 0;; ++t) {
       const int ks = t % kPairKStages, vs = t % kPairVStages;
       if (t >= kPairKStages &&
           !warp_wait(bar_kempty(ks), ((t / kPairKStages) - 1) & 1, wc))
@@ -264,75 +460,39 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       if (t >= kPairVStages &&
           !warp_wait(bar_vempty(vs), ((t / kPairVStages) - 1) & 1, wc))
         break;
-      const TileDesc td = tile_desc(it, t);
-      const uint32_t kf = bar_kfull(ks), vf = bar_vfull(vs);
-      bool contiguous = !td.gather;
-      int key0 = td.key0;
-      if (td.gather) {
-        bool bad = false;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          if (j[r] < 0 || j[r] >= a.L) {
-            bad = true;
-            j[r] = 0;
-          }
-        }
-        if (bad) atomicOr(a.err, kErrBadIndex);
-        // membership masks: bit c of word w <=> row 32w + c belongs to the head.
-        // Lane l holds rows 4l..4l+3, i.e. bits 4(l%8)..4(l%8)+3 of word l/8.
-        uint32_t ma = 0, mb = 0;
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          ma |= (tg[r] & 1u) << r;
-          mb |= ((tg[r] >> 1) & 1u) << r;
-        }
-        ma <<= 4 * (lane & 7);
-        mb <<= 4 * (lane & 7);
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-          ma |= __shfl_xor_sync(0xffffffffu, ma, o);
-          mb |= __shfl_xor_sync(0xffffffffu, mb, o);
-        }
-        if ((lane & 7) == 0) {
-          tags[(vs * 2 + 0) * 4 + (lane >> 3)] = ma;
-          tags[(vs * 2 + 1) * 4 + (lane >> 3)] = mb;
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar_tag0 + 8u * vs);   // publishes this tile's masks
-        const int first = __shfl_sync(0xffffffffu, j[0], 0);
-        const int last = __shfl_sync(0xffffffffu, j[3], 31);
-        // 128 consecutive keys: every lane's four keys are exactly the next
-        // ones (a list entry out of order or repeated keeps the gather path)
-        contiguous = (td.valid == 128) && (last - first == 127) &&
-                     __all_sync(0xffffffffu, j[0] == first + 4 * lane && j[1] == first + 4 * lane + 1 &&
-                                                 j[2] == first + 4 * lane + 2 &&
-                                                 j[3] == first + 4 * lane + 3);
-        key0 = first;
+      const uint32_t desc = nx_desc;
+      // publish the tile: its masks, then its descriptor
+      if ((desc & kDescMasked) && lane < 8) tags[vs * 8 + lane] = nx_mask;
+      __syncwarp();
+      if (lane == 0) {
+        tdesc[vs] = desc;
+        mbar_arrive(bar_tag0 + 8u * vs);
       }
+      const uint32_t kf = bar_kfull(ks), vf = bar_vfull(vs);
       if (lane == 0) {
         mbar_arrive_expect_tx(kf, kTileBytes);
         mbar_arrive_expect_tx(vf, kTileBytes);
       }
       __syncwarp();
-      if (contiguous) {
-        if (lane == 0) {
-          tma_load_2d(s_k(ks), &tm_k, kf, 0, kv_row0 + key0);
-          tma_load_2d(s_k(ks) + kHalfBytes, &tm_k, kf, 64, kv_row0 + key0);
-          tma_load_2d(s_v(vs), &tm_v, vf, 0, kv_row0 + key0);
-          tma_load_2d(s_v(vs) + kHalfBytes, &tm_v, vf, 64, kv_row0 + key0);
-        }
-      } else {
+      if (desc & kDescGather) {
+        // rows 4 l .. 4 l + 3 of the tile from lane l: one gather4 per operand half
         const uint32_t roff = lane * 4u * 128u;
-        tma_gather4(s_k(ks) + roff, &tm_kg, kf, 0, kv_row0 + j[0], kv_row0 + j[1],
-                    kv_row0 + j[2], kv_row0 + j[3]);
-        tma_gather4(s_k(ks) + kHalfBytes + roff, &tm_kg, kf, 64, kv_row0 + j[0],
-                    kv_row0 + j[1], kv_row0 + j[2], kv_row0 + j[3]);
-        tma_gather4(s_v(vs) + roff, &tm_vg, vf, 0, kv_row0 + j[0], kv_row0 + j[1],
-                    kv_row0 + j[2], kv_row0 + j[3]);
-        tma_gather4(s_v(vs) + kHalfBytes + roff, &tm_vg, vf, 64, kv_row0 + j[0],
-                    kv_row0 + j[1], kv_row0 + j[2], kv_row0 + j[3]);
+        tma_gather4(s_k(ks) + roff, &tm_kg, kf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
+        tma_gather4(s_k(ks) + kHalfBytes + roff, &tm_kg, kf, 64, nx_row[0], nx_row[1], nx_row[2],
+                    nx_row[3]);
+        tma_gather4(s_v(vs) + roff, &tm_vg, vf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
+        tma_gather4(s_v(vs) + kHalfBytes + roff, &tm_vg, vf, 64, nx_row[0], nx_row[1], nx_row[2],
+                    nx_row[3]);
+      } else if (lane == 0) {
+        tma_load_2d(s_k(ks), &tm_k, kf, 0, kv_row0 + nx_key0);
+        tma_load_2d(s_k(ks) + kHalfBytes, &tm_k, kf, 64, kv_row0 + nx_key0);
+        tma_load_2d(s_v(vs), &tm_v, vf, 0, kv_row0 + nx_key0);
+        tma_load_2d(s_v(vs) + kHalfBytes, &tm_v, vf, 64, kv_row0 + nx_key0);
       }
+      __syncwarp();
       issued = t + 1;
+      if (desc & kDescLast) break;
+      prepare();
     }
     if (lane == 0) {   // no copy may still be in flight when the CTA exits
       mbar_drain(bar_q, 0, a.wait_ns);
@@ -366,7 +526,7 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                       (t > 0 || kk > 0) ? 1u : 0u);
         }
       };
-      if (ok && T > 0) {
+      if (ok) {
         if ((ok = mbar_wait(bar_kfull(0), 0, wc))) {
           tc_fence_after();
           qk(0, 0);
@@ -374,9 +534,11 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit(bar_kempty(0));
         }
       }
-      for (int t = 0; ok && t < T; ++t) {
+      for (int t = 0; ok; ++t) {
         const int vs = t % kPairVStages;
-        const bool more = t + 1 < T;
+        // tile t's descriptor was written before its loads were armed, and
+        // kfull of tile t has been observed (QK(t) is issued)
+        const bool more = (tdesc[vs] & kDescLast) == 0u;
         // head A: PV(t), then QK(t+1)
         if (!(ok = mbar_wait(bar_pfull0, t & 1, wc))) break;
         if (!(ok = mbar_wait(bar_vfull(vs), (t / kPairVStages) & 1, wc))) break;
@@ -398,6 +560,7 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           mma_commit(bar_kempty((t + 1) % kPairKStages));
         } else {
           mma_commit(bar_odone);
+          break;
         }
       }
       mma_commit(bar_drain);
@@ -416,35 +579,42 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     const float sl2 = a.sl2;
     float m_used = -INFINITY;
     float lsum = 0.f;
-    uint32_t tag_phase = 0u;                   // bit vs: phase of tag barrier vs
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
+    bool last = false;
+    for (int t = 0; !last; ++t) {
       if (!(ok = warp_wait(bar_sfull0 + 8u * hd, t & 1, wc))) break;
       tc_fence_after();
-      const TileDesc td = tile_desc(it, t);
-      const int limit = td.causal ? min(td.valid, r + 1) : td.valid;
-      uint32_t tw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
-      if (td.gather) {
-        const int vs = t % kPairVStages;
-        // tag barrier phases of this slot count the gathered tiles that used it
-        if (!(ok = warp_wait(bar_tag0 + 8u * vs, (tag_phase >> vs) & 1u, wc))) break;
-        tag_phase ^= 1u << vs;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) tw[w] = tags[(vs * 2 + hd) * 4 + w];
-      }
       uint32_t sr[4][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + s_col + 32u * c, sr[c]);
-      tmem_ld_wait();
-      const bool masked = (limit < 128) || ((tw[0] & tw[1] & tw[2] & tw[3]) != 0xffffffffu);
-      if (masked) {
+      // while S comes out of TMEM: the tile's descriptor and masks (every
+      // tile arrives once on its V slot's tag barrier, before its loads)
+      const int vs = t % kPairVStages;
+      if (!(ok = warp_wait(bar_tag0 + 8u * vs, (t / kPairVStages) & 1, wc))) {
+        tmem_ld_wait();
+        break;
+      }
+      const uint32_t dw = tdesc[vs];
+      last = (dw & kDescLast) != 0u;
+      const int valid = static_cast<int>(dw & 0x1FFu);
+      const int limit = (dw & kDescCausal) ? min(valid, r + 1) : valid;
+      uint32_t tw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      if (dw & kDescMasked) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int w = 0; w < 4; ++w) tw[w] = tags[(vs * 2 + hd) * 4 + w];
+      }
+      tmem_ld_wait();
+      // mask the 32-key words with a missing key or past the limit (the head
+      // masks are the same for the whole warp)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (c * 32 + 31 >= limit || tw[c] != 0xffffffffu) {
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const bool v = (c * 32 + e < limit) && ((tw[c] >> e) & 1u);
             if (!v) sr[c][e] = __float_as_uint(-INFINITY);
           }
+        }
       }
       float mxv[8];
 #pragma unroll
@@ -490,15 +660,8 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
           const int c = 2 * h2 + cc;
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float x0 = fmaf(__uint_as_float(sr[c][e]), sl2, neg_m);
-            const float x1 = fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m);
-#if SPA_EXP2_POLY_EVERY > 0
-            const bool poly = ((e >> 1) % SPA_EXP2_POLY_EVERY) == SPA_EXP2_POLY_EVERY - 1;
-#else
-            const bool poly = false;
-#endif
-            const float p0 = poly ? poly_exp2(x0) : fast_exp2(x0);
-            const float p1 = poly ? poly_exp2(x1) : fast_exp2(x1);
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sr[c][e]), sl2, neg_m));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sr[c][e + 1]), sl2, neg_m));
             ps[(e >> 1) & 7] += p0 + p1;
             sr[c][e >> 1] = pack_bf16x2(p0, p1);   // in place: index e/2 was consumed
           }
@@ -510,7 +673,7 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       tc_fence_before();
       mbar_arrive(bar_pfull0 + 8u * hd);
     }
-    if (ok && T > 0) {
+    if (ok) {
       ok = warp_wait(bar_odone, 0, wc);
       if (ok) {
         tc_fence_after();

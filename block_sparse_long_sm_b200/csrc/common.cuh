@@ -21,4 +21,31 @@ __host__ __device__ __forceinline__ long long cap_prefix(long long n, long long 
   return bq * ((n * (n + 1) - q0 * (q0 + 1)) / 2) - cnt * A;
 }
 
+// Candidate key tiles.  The candidates of query block q, [sink, ls_q) with
+// ls_q = (q + 1) * 128 - local a multiple of 128, lie in the 128-key tiles
+// kt0 <= kt < ls_q / 128, kt0 = sink / 128: tmask_tiles(q, c) of them with
+// c = tmask_c(sink, local).  The plan writes one 128-bit mask per such tile
+// (bit k of word w <=> key 128 kt + 32 w + k kept); the masks of block q start
+// at tile tmask_prefix(q, c) of its head's region.
+__host__ __device__ __forceinline__ int tmask_c(int sink, int local) {
+  return 1 - local / 128 - sink / 128;
+}
+__host__ __device__ __forceinline__ int tmask_tiles(int q, int c) { return q + c > 0 ? q + c : 0; }
+__host__ __device__ __forceinline__ long long tmask_prefix(long long n, int c) {
+  const long long m = n + c;
+  return m > 0 ? m * (m - 1) / 2 : 0;
+}
+
+// Tile bitmaps.  Beside the masks the plan writes, per (b, h, query block),
+// three bitmaps over the block's candidate tiles (bit t of word t / 32 <=>
+// candidate tile kt0 + t), each tmask_bit_words(nqb, c) words long:
+// non-empty (some key kept), dense (at least kTileDenseMin keys kept) and
+// full (all 128 keys kept).  The paired attention kernel walks its tiles from
+// them: a tile a head pair keeps densely is loaded whole, the keys of the
+// others are gathered.
+constexpr int kTileDenseMin = 64;
+__host__ __device__ __forceinline__ int tmask_bit_words(int nqb, int c) {
+  return (tmask_tiles(nqb - 1, c) + 31) / 32;
+}
+
 }  // namespace spa

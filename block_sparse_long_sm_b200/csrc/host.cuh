@@ -33,7 +33,11 @@ struct Layout {
   size_t kpart = 0, kmean = 0, q8 = 0, k8 = 0, sq = 0, sk = 0;
   bool paired = false;              // two q heads per attention CTA (Hq / Hkv even)
   bool fused = false;               // ANCHOR: scan and compaction in one kernel
-  size_t pair_counts = 0, pair_lists = 0, pair_split = 0;
+  int tc = 0;                       // candidate-tile constant tmask_c(sink, local)
+  long long tmask_per_head = 0;     // candidate-tile masks per (b, h)
+  size_t tmask = 0;                 // uint4 [B*Hq][tmask_per_head]
+  int tbit_words = 0;               // words of one tile bitmap
+  size_t tbits = 0;                 // uint32 [B*Hq*nqb][3][tbit_words]
   size_t total = 0;
 };
 
@@ -125,13 +129,14 @@ Layout layout_of(const spa_params* p) {
     lo.counts = take(lo.nb * 4);
   }
   lo.paired = (lo.group % 2) == 0;
-  if (lo.paired && p->mode != SPA_MODE_DENSE) {
-    // for the paired attention kernel (opaque scratch): per (b, head pair,
-    // query block) the union size, the split (union entries shared with head
-    // 2p's list) and the tagged union entries from the split on
-    lo.pair_counts = take((lo.nb / 2) * 4);
-    lo.pair_split = take((lo.nb / 2) * 4);
-    lo.pair_lists = take((size_t)(bh / 2) * lo.list_per_head * 4);
+  if (p->mode != SPA_MODE_DENSE) {
+    // one 128-bit mask per (b, h, query block, candidate key tile): the
+    // selection the paired attention kernel reads its tiles from
+    lo.tc = tmask_c(p->sink, p->local);
+    lo.tmask_per_head = tmask_prefix(lo.nqb, lo.tc);
+    lo.tmask = take((size_t)bh * lo.tmask_per_head * 16);
+    lo.tbit_words = lo.nqb > 0 ? tmask_bit_words(lo.nqb, lo.tc) : 0;
+    lo.tbits = take((size_t)lo.nb * 3 * lo.tbit_words * 4);
   }
   lo.total = off;
   lo.ok = true;

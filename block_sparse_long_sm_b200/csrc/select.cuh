@@ -534,12 +534,9 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 // share the kv head, so each K tile feeds both).  The CTA walks every key tile
 // of its candidate range in ascending order and appends each query block's
 // kept keys to the block's list at a running offset, so the lists come out
-// ascending with no intermediate mask.  For a pair it also builds the union
-// of the two heads' kept keys per query block (the paired attention kernel's
-// key list): its size, the number of its entries before the two heads'
-// selections first differ (up to there the union is head 2p's own list),
-// and, from that point on, the entries themselves, each tagged with the heads
-// that kept it (index | in 2p << 30 | in 2p+1 << 31).  Selection groups
+// ascending with no intermediate mask.  It also writes, for every candidate
+// tile of every block, the block's 128 keep bits of that tile (the tile masks
+// the paired attention kernel cuts its tiles from).  Selection groups
 // (step > 1) must lie inside one warp: step a power of two <= 32.
 //
 // Warp 0 loads the pooled-Q tile once and the K tiles (4-stage ring); warp 1
@@ -547,10 +544,11 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 // a TMEM lane quadrant and 32 of the 128 columns (one 32-key word per row).
 // Per key tile the sixteen warps exchange their words through shared memory
 // behind a bounded mbarrier wait, so that every thread knows its row's kept
-// count before its word.  Stores, by density of the warp's 32 words: all keys
-// kept -- one shuffle and one coalesced store of the same 32 values per row;
-// at most 8 keys in every word -- each thread stores its own row's keys; in
-// between -- the rows' (word, list position) pairs are staged and each row
+// count before its word, and the first four warps store each row's four
+// words as its tile mask.  Stores, by density of the warp's 32 words: all
+// keys kept -- one shuffle and one coalesced store of the same 32 values per
+// row; at most 8 keys in every word -- each thread stores its own row's keys;
+// in between -- the rows' (word, list position) pairs are staged and each row
 // with keys is one coalesced store.  CTAs are numbered heaviest first (last M
 // tile first), so the block scheduler fills the GPU longest-job-first.
 constexpr int kSelEpiWarps = 16;
@@ -574,9 +572,11 @@ struct SelectArgs {
   long long list_per_head;
   long long cap_a;
   int* counts;              // [B*Hq*nqb]
-  int* pair_counts;         // [B*Hq/2*nqb] (pairs only)
-  uint32_t* pair_lists;     // [B*Hq/2][list_per_head] tagged union entries (pairs only)
-  int* pair_split;          // [B*Hq/2*nqb]: union entries before the heads first differ
+  uint4* tmask;             // [B*Hq][tmask_per_head] candidate-tile masks
+  long long tmask_per_head;
+  int tc;                   // tmask_c(sink, local)
+  uint32_t* tbits;          // [B*Hq*nqb][3][tbit_words]: non-empty, dense, full tiles
+  int tbit_words;
   uint32_t* err;
   uint64_t wait_ns;
 };
@@ -618,7 +618,6 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
   const int b = bh0 / a.Hq;
   const int kv_row0 = (b * a.Hkv + (bh0 - b * a.Hq) / a.group) * a.L;
   const int BH = a.B * a.Hq;
-  const bool paired = a.heads_per_item == 2;
   // epilogue row of this thread (warps 2-17): TMEM lane r, key word qtr
   const int quad = warp & 3;
   const int qtr = (warp - 2) >> 2;               // key columns [32*qtr, 32*qtr + 32)
@@ -628,8 +627,6 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
   const int bh = bh0 + hs;
   const bool row_valid = warp >= 2 && qb < a.nqb;
   int off = 0;                                   // kept keys written so far (this row)
-  int uoff = 0;                                  // union entries so far (2p+1 rows)
-  int split = -1;                                // union entries before the heads differ
 
   if (threadIdx.x == 0) {
     mbar_init(bar_a, 1);
@@ -718,8 +715,11 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
     // element offset of this row's list inside its head's list region
     const int row_elem = row_valid ? static_cast<int>(cap_prefix(qb, 128, a.cap_a)) : 0;
     int* head_lists = a.lists + (long long)bh * a.list_per_head;    // the same for the warp
-    const bool union_row = paired && hs == 1;     // this thread also writes the pair's union
-    uint32_t* pair_list = paired ? a.pair_lists + (long long)(bh0 >> 1) * a.list_per_head : nullptr;
+    // this row's candidate-tile masks (written by the warps of the first key word)
+    const int n_ct = row_valid ? tmask_tiles(qb, a.tc) : 0;
+    uint4* row_tmask = a.tmask + (long long)bh * a.tmask_per_head + tmask_prefix(qb, a.tc);
+    uint32_t* row_bits = a.tbits + ((long long)bh * a.nqb + qb) * 3 * a.tbit_words;
+    uint32_t occ_acc = 0u, den_acc = 0u, full_acc = 0u;   // this row's tile bits, 32 tiles at a time
     const uint32_t lt = (1u << lane) - 1u;
     uint4* my_stage = stage + (warp - 2) * 32;
     const uint32_t below_q = (1u << qtr) - 1u;  // words of this row before this warp's
@@ -760,34 +760,22 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
         before += ((below_q >> q) & 1u) ? c : 0;
         total += c;
       }
-      uint32_t awq = 0u;                              // head 2p's word (2p+1 rows)
-      int ubefore = 0, utotal = 0;
-      bool write_union = false;
-      if (union_row) {
-        const uint4 av = x_words[xs * 128 + (r - 64)];
-        const uint32_t* aw = &av.x;
-        // While the two heads agree, the union is head 2p's list; union
-        // entries are written from the first differing word on.
-        const bool diverged = split >= 0;
-        int first_diff = 4, ucount = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int cu = __popc(aw[q] | mw[q]);
-          if (first_diff == 4 && aw[q] != mw[q]) {
-            first_diff = q;
-            if (!diverged) split = uoff + ucount;
-          }
-          ucount += cu;
-          ubefore += ((below_q >> q) & 1u) ? cu : 0;
-          utotal += cu;
+      if (qtr == 0 && t < n_ct) {
+        row_tmask[t] = mine;
+        const uint32_t bit = 1u << (t & 31);
+        if (total > 0) occ_acc |= bit;
+        if (total >= kTileDenseMin) den_acc |= bit;
+        if (total == 128) full_acc |= bit;
+        if ((t & 31) == 31 || t == n_ct - 1) {
+          row_bits[t >> 5] = occ_acc;
+          row_bits[a.tbit_words + (t >> 5)] = den_acc;
+          row_bits[2 * a.tbit_words + (t >> 5)] = full_acc;
+          occ_acc = den_acc = full_acc = 0u;
         }
-        write_union = diverged || first_diff <= qtr;
-        awq = qtr == 0 ? av.x : qtr == 1 ? av.y : qtr == 2 ? av.z : av.w;
       }
       // append.  When every row of the warp keeps all 32 keys of its word (the
       // dense case), every row stores the same 32 values: one shuffle and one
-      // coalesced store per row.  Otherwise, and for union entries, stage
-      // (word, list position, head 2p's word, union position or none) and
+      // coalesced store per row.  Otherwise stage (word, list position) and
       // store each row's set bits.
       const int key = key0 + lane;
       const int pos = row_elem + off + before;
@@ -797,60 +785,35 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) hl[__shfl_sync(0xffffffffu, pos, j)] = key;
       }
-      // rows with something to store: own keys (unless stored above) or union entries
-      const uint32_t need = __ballot_sync(
-          0xffffffffu, (!dense && w != 0u) || (write_union && (w | awq) != 0u));
+      // rows with keys still to store
+      const uint32_t need = __ballot_sync(0xffffffffu, !dense && w != 0u);
       // few keys per row (every word of the warp at most 8 bits): each thread
       // stores its own row's keys, one per step, instead of a warp-wide store
       // per row
-      const uint32_t uw = write_union ? (w | awq) : 0u;
-      const bool sparse = need != 0u &&
-          __reduce_max_sync(0xffffffffu, max(dense ? 0 : __popc(w), __popc(uw))) <= 8;
+      const bool sparse = need != 0u && __reduce_max_sync(0xffffffffu, __popc(w)) <= 8;
       if (sparse) {
-        uint32_t rem = dense ? 0u : w, urem = uw;
-        int k = 0, ku = 0;
-        const int upos = row_elem + uoff + ubefore;
-        while (__any_sync(0xffffffffu, (rem | urem) != 0u)) {
+        uint32_t rem = w;
+        int k = 0;
+        while (__any_sync(0xffffffffu, rem != 0u)) {
           if (rem) {
             head_lists[pos + k++] = key0 + __ffs(rem) - 1;
             rem &= rem - 1u;
           }
-          if (urem) {
-            const int e = __ffs(urem) - 1;
-            const uint32_t tag = (((awq >> e) & 1u) << 30) | (((w >> e) & 1u) << 31);
-            pair_list[upos + ku++] = static_cast<uint32_t>(key0 + e) | tag;
-            urem &= urem - 1u;
-          }
         }
       } else if (need) {
-        my_stage[lane] = make_uint4(w, static_cast<uint32_t>(pos), awq,
-                                    write_union ? static_cast<uint32_t>(row_elem + uoff + ubefore)
-                                                : 0xffffffffu);
+        my_stage[lane] = make_uint4(w, static_cast<uint32_t>(pos), 0u, 0u);
         __syncwarp();
         for (uint32_t rows = need; rows; rows &= rows - 1u) {
           const int j = __ffs(rows) - 1;
           const uint4 v = my_stage[j];
-          if (!dense) {                               // warp-uniform
-            if (v.x == 0xffffffffu) {
-              head_lists[static_cast<int>(v.y) + lane] = key;
-            } else if (v.x != 0u) {
-              if ((v.x >> lane) & 1u) head_lists[static_cast<int>(v.y) + __popc(v.x & lt)] = key;
-            }
-          }
-          if (v.w != 0xffffffffu) {                   // warp-uniform
-            const uint32_t u = v.x | v.z;
-            const uint32_t tag = (((v.z >> lane) & 1u) << 30) | (((v.x >> lane) & 1u) << 31);
-            if (u == 0xffffffffu) {
-              pair_list[static_cast<int>(v.w) + lane] = static_cast<uint32_t>(key) | tag;
-            } else if (u != 0u) {
-              if ((u >> lane) & 1u)
-                pair_list[static_cast<int>(v.w) + __popc(u & lt)] = static_cast<uint32_t>(key) | tag;
-            }
+          if (v.x == 0xffffffffu) {
+            head_lists[static_cast<int>(v.y) + lane] = key;
+          } else if ((v.x >> lane) & 1u) {
+            head_lists[static_cast<int>(v.y) + __popc(v.x & lt)] = key;
           }
         }
         __syncwarp();
       }
-      uoff += utotal;
       off += total;
     }
   }
@@ -858,13 +821,7 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
   __syncthreads();
   tc_fence_after();
   // written even after an abort: a count never exceeds its block's capacity
-  if (warp >= 2 && qtr == 0 && row_valid) {
-    a.counts[(long long)bh * a.nqb + qb] = off;
-    if (paired && hs == 1) {
-      a.pair_counts[(long long)(bh0 >> 1) * a.nqb + qb] = uoff;
-      a.pair_split[(long long)(bh0 >> 1) * a.nqb + qb] = split < 0 ? uoff : split;
-    }
-  }
+  if (warp >= 2 && qtr == 0 && row_valid) a.counts[(long long)bh * a.nqb + qb] = off;
   if (warp == 1) tmem_dealloc(tmem, 512);
 }
 
@@ -961,157 +918,86 @@ compact_kernel(const CompactArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// two heads' bitmasks -> both heads' lists + one tagged union list
+// bitmask -> candidate-tile masks
 // ---------------------------------------------------------------------------
-// For the paired attention kernel (two q heads of one GQA group share every
-// K/V tile).  One pass over the two bitmask rows writes head A's and head
-// B's ascending lists and counts (the documented per-head output, exactly as
-// compact_kernel would) and the union list, whose entries are
-// index | (kept by head 2p) << 30 | (kept by head 2p+1) << 31.
-struct PairCompactArgs {
-  int nqb, heads_q, sink, local, unit, step;
-  const uint32_t* mask;     // [B*Hq*nqb][nwords]
+// The bitmask paths (SALE, and ANCHOR when step is not a power of two <= 32)
+// write the tile masks the paired attention kernel reads: for query block qb
+// and candidate tile kt (kt0 <= kt < ls / 128), bit k of word w is set when
+// key 128 kt + 32 w + k lies in [sink, ls) and its unit (the key, or its key
+// block in SALE mode) is kept by some block of the selection group, exactly
+// the keys compact_kernel lists; and the block's three tile bitmaps.  One
+// CTA per block row, one thread per tile.
+struct TileMaskArgs {
+  int nqb, sink, local, unit, step, tc;
+  const uint32_t* mask;     // [B*Hq*nqb][nwords] over units
   int nwords;
-  int* lists;               // per-head lists (as compact_kernel)
-  int* counts;              // per-head counts
-  uint32_t* pair_lists;     // [B*Hq/2][per_head] tagged entries
-  long long list_per_head;
-  long long cap_a;
-  int* pair_counts;         // [B*Hq/2*nqb]
-  int* pair_split;          // [B*Hq/2*nqb]: union entries before the heads first differ
+  uint4* tmask;             // [B*Hq][tmask_per_head]
+  long long tmask_per_head;
+  uint32_t* tbits;          // [B*Hq*nqb][3][tbit_words]
+  int tbit_words;
 };
 
-__global__ void __launch_bounds__(kCompactThreads)
-pair_compact_kernel(const PairCompactArgs a) {
-  const int row = blockIdx.x;                       // (b, pair, qb)
-  const int pair = row / a.nqb, qb = row - (row / a.nqb) * a.nqb;
-  const int b = pair / (a.heads_q / 2), pp = pair - b * (a.heads_q / 2);
-  const int bhA = b * a.heads_q + 2 * pp;
-  const long long rowA = (long long)bhA * a.nqb + qb;
-  const long long rowB = rowA + a.nqb;
+__global__ void __launch_bounds__(128) tile_mask_kernel(const TileMaskArgs a) {
+  const int row = blockIdx.x;
+  const int bh = row / a.nqb, qb = row - bh * a.nqb;
   const int ls = max(0, (qb + 1) * 128 - a.local);
-  const int bit_lo = a.sink / a.unit;
-  const int bit_hi = max(a.sink, ls) / a.unit;
-  const int w_lo = bit_lo / 32;
-  const int w_hi = bit_hi > bit_lo ? (bit_hi + 31) / 32 : w_lo;
-  const int n = w_hi - w_lo;
+  const int n_ct = tmask_tiles(qb, a.tc);
+  const int kt0 = a.sink / 128;
   const int g0 = (qb / a.step) * a.step;
   const int g1 = min(g0 + a.step, a.nqb);
-  const uint32_t* mA0 = a.mask + (rowA - qb) * a.nwords;     // block 0 of head A
-  const uint32_t* mB0 = a.mask + (rowB - qb) * a.nwords;
-  auto words_at = [&](int w, uint32_t& wa, uint32_t& wb) {
-    if (a.step == 1) {
-      wa = mA0[(long long)qb * a.nwords + w];
-      wb = mB0[(long long)qb * a.nwords + w];
-      return;
-    }
-    wa = 0u;
-    wb = 0u;
+  const int lane = threadIdx.x & 31;
+  const uint32_t* mrow0 = a.mask + ((long long)row - qb) * a.nwords;   // block 0 of this head
+  // bit u of the group's selection (each row read only inside its own range)
+  auto unit_kept = [&](int u) -> uint32_t {
+    uint32_t v = 0;
     for (int b2 = g0; b2 < g1; ++b2) {
       const int ls2 = max(0, (b2 + 1) * 128 - a.local);
       const int hi2 = max(a.sink, ls2) / a.unit;
-      if (w < (hi2 + 31) / 32) {
-        wa |= mA0[(long long)b2 * a.nwords + w];
-        wb |= mB0[(long long)b2 * a.nwords + w];
-      }
+      if (u >= a.sink / a.unit && u < hi2) v |= mrow0[(long long)b2 * a.nwords + u / 32] >> (u % 32);
     }
+    return v & 1u;
   };
-  const long long off = cap_prefix(qb, 128, a.cap_a) / a.unit;
-  int* outA = a.lists + (long long)bhA * a.list_per_head + off;
-  int* outB = outA + a.list_per_head;
-  uint32_t* outU = a.pair_lists + (long long)pair * a.list_per_head + off;
-
-  __shared__ int warp_cnt[3][kCompactThreads / 32];
-  __shared__ int warp_base[3][kCompactThreads / 32];
-  __shared__ int warp_diff[kCompactThreads / 32];
-  __shared__ int first_diff;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nw = kCompactThreads / 32;
-  const int seg = (((n + nw - 1) / nw) + 31) & ~31;
-  const int s_lo = w_lo + warp * seg;
-  const int s_hi = min(s_lo + seg, w_hi);
-  int ca = 0, cb = 0, cu = 0, diff = 0x7fffffff;    // diff: first word where the heads differ
-  for (int w = s_lo + lane; w < s_hi; w += 32) {
-    uint32_t wa, wb;
-    words_at(w, wa, wb);
-    ca += __popc(wa);
-    cb += __popc(wb);
-    cu += __popc(wa | wb);
-    if (wa != wb) diff = min(diff, w);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    ca += __shfl_xor_sync(0xffffffffu, ca, o);
-    cb += __shfl_xor_sync(0xffffffffu, cb, o);
-    cu += __shfl_xor_sync(0xffffffffu, cu, o);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) diff = min(diff, __shfl_xor_sync(0xffffffffu, diff, o));
-  if (lane == 0) {
-    warp_cnt[0][warp] = ca;
-    warp_cnt[1][warp] = cb;
-    warp_cnt[2][warp] = cu;
-    warp_diff[warp] = diff;
-  }
-  __syncthreads();
-  if (threadIdx.x < 3) {
-    int run = 0;
-    for (int i = 0; i < nw; ++i) {
-      warp_base[threadIdx.x][i] = run;
-      run += warp_cnt[threadIdx.x][i];
-    }
-    if (threadIdx.x == 0) a.counts[rowA] = run;
-    if (threadIdx.x == 1) a.counts[rowB] = run;
-    if (threadIdx.x == 2) {
-      int m = 0x7fffffff;
-      for (int i = 0; i < nw; ++i) m = min(m, warp_diff[i]);
-      first_diff = m;
-      a.pair_counts[row] = run;
-      if (m == 0x7fffffff) a.pair_split[row] = run;            // the heads agree throughout
-    }
-  }
-  __syncthreads();
-  const int fd = first_diff;
-  int base_a = warp_base[0][warp], base_b = warp_base[1][warp], base_u = warp_base[2][warp];
-  const uint32_t lt = (1u << lane) - 1u;
-  auto scan = [&](int v) {
-    int incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int t = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += t;
-    }
-    return incl;
-  };
-  for (int w0 = s_lo; w0 < s_hi; w0 += 32) {
-    uint32_t wa = 0u, wb = 0u;
-    if (w0 + lane < s_hi) words_at(w0 + lane, wa, wb);
-    const uint32_t wu = wa | wb;
-    const int ia = scan(__popc(wa)), ib = scan(__popc(wb)), iu = scan(__popc(wu));
-    const int ea = ia - __popc(wa), eb = ib - __popc(wb), eu = iu - __popc(wu);
-    for (int j = 0; j < 32; ++j) {
-      // every shuffle is executed by the whole warp, before any lane-dependent branch
-      const uint32_t uj = __shfl_sync(0xffffffffu, wu, j);
-      if (uj == 0u) continue;                         // warp-uniform
-      const uint32_t aj = __shfl_sync(0xffffffffu, wa, j);
-      const uint32_t bj = __shfl_sync(0xffffffffu, wb, j);
-      const int ou = __shfl_sync(0xffffffffu, eu, j);
-      const int oa = __shfl_sync(0xffffffffu, ea, j);
-      const int ob = __shfl_sync(0xffffffffu, eb, j);
-      const int key = 32 * (w0 + j) + lane;
-      // union entries from the first word where the heads differ (before
-      // it the union is head A's list); that word's offset is the split
-      if (w0 + j == fd && lane == 0) a.pair_split[row] = base_u + ou;
-      if (w0 + j >= fd && ((uj >> lane) & 1u)) {
-        const uint32_t tag = (((aj >> lane) & 1u) << 30) | (((bj >> lane) & 1u) << 31);
-        outU[base_u + ou + __popc(uj & lt)] = static_cast<uint32_t>(key) | tag;
+  uint4* out = a.tmask + (long long)bh * a.tmask_per_head + tmask_prefix(qb, a.tc);
+  uint32_t* bits = a.tbits + (long long)row * 3 * a.tbit_words;
+  // one tile per thread; a warp covers 32 consecutive tiles (one bitmap word)
+  for (int t0 = threadIdx.x & ~31; t0 < n_ct; t0 += blockDim.x) {
+    const int t = t0 + lane;
+    uint32_t w4[4] = {0u, 0u, 0u, 0u};
+    if (t < n_ct) {
+      for (int wi = 0; wi < 4; ++wi) {
+        const int key0 = 128 * (kt0 + t) + 32 * wi;
+        uint32_t word = 0;
+        if (a.unit == 1) {
+          // the 32 keys are one bitmask word; a row's words inside its range
+          // are written whole (compact_kernel reads them the same way)
+          for (int b2 = g0; b2 < g1; ++b2) {
+            const int ls2 = max(0, (b2 + 1) * 128 - a.local);
+            if (key0 / 32 < (max(a.sink, ls2) + 31) / 32)
+              word |= mrow0[(long long)b2 * a.nwords + key0 / 32];
+          }
+        } else {
+          for (int k = 0; k < 32; k += min(a.unit, 32)) {
+            const uint32_t run = a.unit >= 32 ? 0xffffffffu : ((1u << a.unit) - 1u);
+            if (unit_kept((key0 + k) / a.unit)) word |= run << k;
+          }
+        }
+        // the block's candidates [sink, ls)
+        const int lo = max(a.sink - key0, 0), hi = min(ls - key0, 32);
+        uint32_t range = 0;
+        if (hi > lo) range = (hi - lo >= 32 ? 0xffffffffu : ((1u << (hi - lo)) - 1u)) << lo;
+        w4[wi] = word & range;
       }
-      if ((aj >> lane) & 1u) outA[base_a + oa + __popc(aj & lt)] = key;
-      if ((bj >> lane) & 1u) outB[base_b + ob + __popc(bj & lt)] = key;
+      out[t] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
-    base_a += __shfl_sync(0xffffffffu, ia, 31);
-    base_b += __shfl_sync(0xffffffffu, ib, 31);
-    base_u += __shfl_sync(0xffffffffu, iu, 31);
+    const int c = __popc(w4[0]) + __popc(w4[1]) + __popc(w4[2]) + __popc(w4[3]);
+    const uint32_t occ = __ballot_sync(0xffffffffu, c > 0);
+    const uint32_t den = __ballot_sync(0xffffffffu, c >= kTileDenseMin);
+    const uint32_t full = __ballot_sync(0xffffffffu, c == 128);
+    if (lane == 0) {
+      bits[t0 >> 5] = occ;
+      bits[a.tbit_words + (t0 >> 5)] = den;
+      bits[2 * a.tbit_words + (t0 >> 5)] = full;
+    }
   }
 }
 

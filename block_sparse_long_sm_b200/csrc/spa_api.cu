@@ -107,10 +107,8 @@ SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const
                     reinterpret_cast<const float*>(ws + lo.xbar),
                     reinterpret_cast<int*>(ws + lo.lists), lo.list_per_head, lo.cap_a,
                     reinterpret_cast<int*>(ws + lo.counts),
-                    lo.paired ? reinterpret_cast<int*>(ws + lo.pair_counts) : nullptr,
-                    lo.paired ? reinterpret_cast<uint32_t*>(ws + lo.pair_lists) : nullptr,
-                    lo.paired ? reinterpret_cast<int*>(ws + lo.pair_split) : nullptr, err,
-                    wait_ns(p)};
+                    reinterpret_cast<uint4*>(ws + lo.tmask), lo.tmask_per_head, lo.tc,
+                    reinterpret_cast<uint32_t*>(ws + lo.tbits), lo.tbit_words, err, wait_ns(p)};
       if (set_smem(stripe_select_kernel, kSelSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
       stripe_select_kernel<<<(unsigned)(n_mt * (BH / hpi)), kSelThreads, kSelSmemBytes, stream>>>(
           tqsel, tk, sa);
@@ -162,23 +160,20 @@ SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const
         tq8, tk8, sa);
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   }
-  if (lo.paired) {
-    // one pass writes both heads' lists, their union's size and split, and
-    // the tagged union entries from the first difference on
-    PairCompactArgs pc{lo.nqb, Hq, p->sink, p->local, lo.unit, p->step,
-                       reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
-                       reinterpret_cast<int*>(ws + lo.lists), reinterpret_cast<int*>(ws + lo.counts),
-                       reinterpret_cast<uint32_t*>(ws + lo.pair_lists), lo.list_per_head, lo.cap_a,
-                       reinterpret_cast<int*>(ws + lo.pair_counts),
-                       reinterpret_cast<int*>(ws + lo.pair_split)};
-    pair_compact_kernel<<<(unsigned)(lo.nb / 2), kCompactThreads, 0, stream>>>(pc);
-    if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
-  } else {
+  {
     CompactArgs ca{(int)lo.nb, lo.nqb, L, p->sink, p->local, lo.unit, p->step,
                    reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
                    reinterpret_cast<int*>(ws + lo.lists), lo.list_per_head, lo.cap_a,
                    reinterpret_cast<int*>(ws + lo.counts)};
     compact_kernel<<<(unsigned)lo.nb, kCompactThreads, 0, stream>>>(ca);
+    if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
+  }
+  if (lo.tmask_per_head > 0) {
+    TileMaskArgs ta{lo.nqb, p->sink, p->local, lo.unit, p->step, lo.tc,
+                    reinterpret_cast<const uint32_t*>(ws + lo.mask), lo.nwords,
+                    reinterpret_cast<uint4*>(ws + lo.tmask), lo.tmask_per_head,
+                    reinterpret_cast<uint32_t*>(ws + lo.tbits), lo.tbit_words};
+    tile_mask_kernel<<<(unsigned)lo.nb, 128, 0, stream>>>(ta);
     if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   }
   return SPA_OK;

@@ -7,8 +7,7 @@
 #include "../../include/spa.h"
 #include "attn.cuh"
 #include "attn_pair.cuh"
-#include "attn_pair_fp8.cuh"
-#include "attn_pair_win.cuh"
+#include "attn_fp8.cuh"
 #include "host.cuh"
 
 namespace {
@@ -37,7 +36,7 @@ SPA_API spa_status sparse_prefill_attn(const spa_params* p, const void* q, const
       !map_2d(&tv, kBF16, 2, v, 128, BKV * L, 64, 128, kSW128) ||
       !map_2d(&tvg, kBF16, 2, v, 128, BKV * L, 64, 1, kSW128))
     return SPA_ERR_CUDA;
-  AttnArgs aa;
+  AttnArgs aa{};
   aa.B = B; aa.Hq = Hq; aa.Hkv = Hkv; aa.L = L; aa.nqb = lo.nqb; aa.group = lo.group;
   aa.sink = p->sink; aa.local = p->local;
   aa.mode = p->mode == SPA_MODE_ANCHOR ? kModeAnchor : (p->mode == SPA_MODE_SALE ? kModeSale : kModeDense);
@@ -48,20 +47,19 @@ SPA_API spa_status sparse_prefill_attn(const spa_params* p, const void* q, const
   aa.list_per_head = lo.list_per_head;
   aa.cap_a = lo.cap_a;
   aa.list_unit = lo.unit;
-  aa.pair_counts = reinterpret_cast<const int*>(ws + lo.pair_counts);
-  aa.pair_lists = reinterpret_cast<const uint32_t*>(ws + lo.pair_lists);
-  aa.pair_split = reinterpret_cast<const int*>(ws + lo.pair_split);
-  aa.pair_per_head = lo.list_per_head;
+  aa.tmask = reinterpret_cast<const uint4*>(ws + lo.tmask);
+  aa.tmask_per_head = lo.tmask_per_head;
+  aa.tc = lo.tc;
+  aa.tbits = reinterpret_cast<const uint32_t*>(ws + lo.tbits);
+  aa.tbit_words = lo.tbit_words;
+  aa.k = static_cast<const __nv_bfloat16*>(k);
+  aa.v = static_cast<const __nv_bfloat16*>(v);
   aa.o = static_cast<__nv_bfloat16*>(o);
   aa.lse = lse;
   aa.err = reinterpret_cast<uint32_t*>(ws);
   aa.wait_ns = wait_ns(p);
   aa.debug = p->debug_flags;
-  if (lo.paired && (p->debug_flags & SPA_DEBUG_WINDOW_TILES)) {
-    if (set_smem(sparse_attn_pair_win_kernel, kPairSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
-    sparse_attn_pair_win_kernel<<<(unsigned)(lo.nb / 2), kPairThreads, kPairSmemBytes, stream>>>(
-        tq, tk, tkg, tv, tvg, aa);
-  } else if (lo.paired) {
+  if (lo.paired) {
     if (set_smem(sparse_attn_pair_kernel, kPairSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
     sparse_attn_pair_kernel<<<(unsigned)(lo.nb / 2), kPairThreads, kPairSmemBytes, stream>>>(
         tq, tk, tkg, tv, tvg, aa);
@@ -110,31 +108,9 @@ SPA_API spa_status sparse_prefill_attn_fp8(const spa_params* p, const void* q8, 
   a.lse = lse;
   a.err = reinterpret_cast<uint32_t*>(ws);
   a.wait_ns = wait_ns(p);
-  if (lo.paired && p->mode != SPA_MODE_DENSE) {
-    // two q heads per CTA over the pair's union lists
-    PairF8Args pa;
-    pa.base.B = B; pa.base.Hq = Hq; pa.base.Hkv = Hkv; pa.base.L = L; pa.base.nqb = lo.nqb;
-    pa.base.group = lo.group; pa.base.sink = p->sink; pa.base.local = p->local;
-    pa.base.mode = a.g.mode; pa.base.bk = p->block_k;
-    pa.base.sl2 = a.sl2;
-    pa.base.counts = a.g.counts; pa.base.lists = a.g.lists;
-    pa.base.list_per_head = lo.list_per_head; pa.base.cap_a = lo.cap_a;
-    pa.base.list_unit = lo.unit;
-    pa.base.pair_counts = reinterpret_cast<const int*>(ws + lo.pair_counts);
-    pa.base.pair_lists = reinterpret_cast<const uint32_t*>(ws + lo.pair_lists);
-    pa.base.pair_split = reinterpret_cast<const int*>(ws + lo.pair_split);
-    pa.base.pair_per_head = lo.list_per_head;
-    pa.base.o = a.o; pa.base.lse = lse; pa.base.err = a.err; pa.base.wait_ns = a.wait_ns;
-    pa.base.debug = 0;
-    pa.qs = a.qs; pa.ks = a.ks; pa.vs = a.vs; pa.kmean = a.kmean; pa.scale = a.scale;
-    if (set_smem(sparse_attn_pair_fp8_kernel, kPF8SmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
-    sparse_attn_pair_fp8_kernel<<<(unsigned)(lo.nb / 2), kPairThreads, kPF8SmemBytes, stream>>>(
-        tq, tk, tkg, tv, tvg, pa);
-  } else {
-    if (set_smem(sparse_attn_fp8_kernel, kF8SmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
-    sparse_attn_fp8_kernel<<<(unsigned)lo.nb, kF8Threads, kF8SmemBytes, stream>>>(tq, tk, tkg,
-                                                                                 tv, tvg, a);
-  }
+  if (set_smem(sparse_attn_fp8_kernel, kF8SmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
+  sparse_attn_fp8_kernel<<<(unsigned)lo.nb, kF8Threads, kF8SmemBytes, stream>>>(tq, tk, tkg, tv,
+                                                                               tvg, a);
   if (cudaGetLastError() != cudaSuccess) return SPA_ERR_CUDA;
   return SPA_OK;
 }

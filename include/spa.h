@@ -119,11 +119,6 @@ typedef struct {
  * the kernel then records SPA_ERR_TIMEOUT and returns without faulting. */
 #define SPA_DEBUG_STALL_ATTN 0x1u
 
-/* Variant switch (paired attention, Hq / Hkv even): cut the selected keys
- * into 128-key windows loaded contiguously with the absent keys masked,
- * where a window holds at least 96 selected keys, instead of gathering every
- * tile of 128 selected keys row by row.  Same result up to rounding. */
-#define SPA_DEBUG_WINDOW_TILES 0x2u
 
 typedef struct {
   uint32_t error_bits;       /* device error word: bit0 timeout, bit1 bad index */

@@ -84,13 +84,13 @@ def test_workspace_bytes_cover_documented_regions():
             unit = 32 if mode == "sale" else 1
             per_head = binding.cap_prefix(nqb, 256, 128) // unit if mode != "dense" else 0
             assert n >= lists_at + 4 * 32 * per_head
-    # the 128K Llama layer: per-head lists (~8.55 GB), the head pairs' tagged
-    # union lists (~4.28 GB) and small scratch; the bitmask (0.54 GB) only when
-    # the selection groups do not fit a warp
+    # the 128K Llama layer: per-head lists (~8.55 GB), the candidate-tile
+    # masks (16 B per candidate tile: ~0.27 GB) and small scratch; the bitmask
+    # (0.54 GB) only when the selection groups do not fit a warp
     p = spa.make_params(1, 32, 8, 131072)
-    assert 12.8e9 < spa.sparse_prefill_workspace_bytes(p) < 12.9e9
+    assert 8.8e9 < spa.sparse_prefill_workspace_bytes(p) < 8.9e9
     p = spa.make_params(1, 32, 8, 131072, step=3)
-    assert 13.35e9 < spa.sparse_prefill_workspace_bytes(p) < 13.45e9
+    assert 9.35e9 < spa.sparse_prefill_workspace_bytes(p) < 9.45e9
 
 
 def test_shard_units_partition():
