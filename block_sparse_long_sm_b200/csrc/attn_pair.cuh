@@ -15,12 +15,15 @@
 //                    time (the last one padded), copied row by row;
 //   local tiles      keys [ls, row0 + 128), contiguous; the last one is the
 //                    causally masked diagonal.
+// They are loaded in the order sink, dense, local before the diagonal,
+// gathered, diagonal: the gathered tiles' keys are being collected while the
+// first tiles load, and the diagonal is always the last tile.
 // The candidate tiles come from the plan's tile masks (one 128-bit keep mask
 // per head, query block and candidate tile), so the kernel reads 32 bytes of
 // selection per 128 candidate keys and no index list.  Attention over a key
 // set does not depend on the order of its tiles.
 //
-// Roles (384 threads, 3 warpgroups; warps 10 and 11 have no role):
+// Roles (384 threads, 3 warpgroups):
 //   warp 8       producer: Q of both heads once; per tile it picks the keys
 //                (sink, dense, gathered or local), publishes a descriptor and
 //                the two heads' column masks through the tile's tag barrier,
@@ -28,7 +31,10 @@
 //                stages: contiguous tiles as two 64-column boxes per operand.
 //                Gathered tiles are copied row by row with TMA gather4 (four
 //                rows per instruction, issued by the 32 lanes);
-//   warp 9       TMEM allocation and the single MMA-issuing thread, in the
+//   warps 10,11  collectors: each turns the masks of half of the sparse
+//                candidate tiles (bitmap words of one parity) into gathered
+//                tiles of 128 keys and their column masks, one buffer ahead
+//                of the producer;//   warp 9       TMEM allocation and the single MMA-issuing thread, in the
 //                order PV_A(t), QK_A(t+1), PV_B(t), QK_B(t+1), so the tensor
 //                core works on one head while the other head's softmax runs.
 //                P is written by the softmax into the first 64 columns of its
@@ -54,7 +60,7 @@ namespace spa {
 constexpr int kPairKStages = 3;
 constexpr int kPairVStages = 2;
 constexpr int kPairThreads = 384;   // 3 warpgroups: softmax A, softmax B, load + MMA
-constexpr uint32_t kPairBarBytes = 1024u;   // barriers, masks, descriptors, staged keys
+constexpr uint32_t kPairBarBytes = 2048u;   // barriers, masks, descriptors, collected keys
 constexpr uint32_t kPairSmemBytes =
     1024u + 2u * kTileBytes + (kPairKStages + kPairVStages) * kTileBytes + kPairBarBytes;
 static_assert(kPairSmemBytes <= 232448u, "more shared memory than a CTA may use");
@@ -173,10 +179,16 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
   // and the kDesc* flags; written by the producer before it arrives on the
   // slot's tag barrier
   uint32_t* tdesc = reinterpret_cast<uint32_t*>(bar_area + 336);
-  // the next gathered tile's keys, row by row (index | head A kept it << 30 |
-  // head B kept it << 31), while the producer collects them; padding rows
-  // repeat row 0's key with neither head's bit
-  uint32_t* stage = reinterpret_cast<uint32_t*>(bar_area + 512);   // [128]
+  // Gathered tiles are collected by warps 10 and 11, one buffer each: the
+  // keys row by row (index | head A kept it << 30 | head B kept it << 31;
+  // padding rows repeat row 0's key with neither head's bit), the tile's
+  // column masks (words 0-3 head A, 4-7 head B) and the number of keys (0:
+  // that collector has no more).
+  const uint32_t bar_cfull0 = bar_sfull0 + 72u;    // [2] collector -> producer
+  const uint32_t bar_cempty0 = bar_sfull0 + 88u;   // [2] producer -> collector
+  uint32_t* ccount = tdesc + 2;                                     // [2]
+  uint32_t* cmask = reinterpret_cast<uint32_t*>(bar_area + 384);    // [2][8]
+  uint32_t* cbuf = reinterpret_cast<uint32_t*>(bar_area + 512);     // [2][128]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -196,6 +208,10 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       mbar_init(bar_pfull0 + 8u * i, 128);
     }
     for (int st = 0; st < kPairVStages; ++st) mbar_init(bar_tag0 + 8u * st, 1);
+    for (int c = 0; c < 2; ++c) {
+      mbar_init(bar_cfull0 + 8u * c, 1);
+      mbar_init(bar_cempty0 + 8u * c, 1);
+    }
     mbar_init(bar_odone, 1);
     mbar_init(bar_drain, 1);
     mbar_init(bar_stall, 1);
@@ -279,16 +295,220 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       full = ((fbits >> b) & 1u) != 0u;
       return 32 * (32 * dchunk + dwi) + b;
     };
-    // Gathered tiles: the keys of the tiles that are non-empty and not dense,
-    // taken a window at a time (the sparse tiles of one bitmap word, lane j
-    // holding the j-th), the next window's masks loaded ahead.
+    if (nw > 0) load_dense_chunk(0);
+    // Tile order: sink, dense, the local tiles before the diagonal, gathered
+    // (the collectors fill their first buffers meanwhile), the diagonal.
+    int phase = 0;        // 0 sink, 1 dense, 2 early local, 3 gathered, 4 diagonal
+    int n_sink = 0, n_loc = 0;
+    int col = 0;                                   // collector to take the next gathered tile from
+    int taken0 = 0, taken1 = 0;                    // buffers taken from each collector
+    bool cdone0 = false, cdone1 = false;
+    // The next tile, prepared while the previous tile's loads are in flight:
+    // its descriptor, its first key (contiguous tiles), lane l's four rows
+    // 4 l .. 4 l + 3 (gathered tiles) and, in lanes 0-7, word l of the two
+    // heads' column masks (0-3 head A, 4-7 head B).
+    uint32_t nx_desc = 0u;
+    int nx_key0 = 0;
+    int nx_row[4] = {0, 0, 0, 0};
+    uint32_t nx_mask = 0u;
+    auto prepare = [&]() -> bool {
+      nx_desc = 0u;
+      if (phase == 0) {
+        if (n_sink < it.n_sink_t) {
+          nx_key0 = 128 * n_sink++;
+          nx_desc = static_cast<uint32_t>(min(128, it.sink_end - nx_key0));
+          return true;
+        }
+        phase = 1;
+      }
+      if (phase == 1) {
+        bool full = false;
+        const int j = nw > 0 ? next_dense(full) : -1;
+        if (j >= 0) {
+          if (!full && lane < 8)
+            nx_mask = reinterpret_cast<const uint32_t*>(lane < 4 ? pi.ma + j : pi.mb + j)[lane & 3];
+          nx_key0 = 128 * (kt0 + j);
+          nx_desc = 128u | (full ? 0u : kDescMasked);
+          return true;
+        }
+        phase = 2;
+      }
+      if (phase == 2) {
+        if (n_loc + 1 < it.n_loc_t) {
+          nx_key0 = it.loc_start + 128 * n_loc++;
+          nx_desc = static_cast<uint32_t>(min(128, it.le - nx_key0)) |
+                    (nx_key0 == it.row0 ? kDescCausal : 0u);
+          return true;
+        }
+        phase = 3;
+      }
+      if (phase == 3) {
+        // the gathered tiles the two collector warps prepare, taken in turn
+        while (!(cdone0 && cdone1)) {
+          if (col == 0 ? cdone0 : cdone1) col ^= 1;
+          const int c = col;
+          const int tk = c == 0 ? taken0++ : taken1++;
+          if (!warp_wait(bar_cfull0 + 8u * c, tk & 1, wc)) return false;
+          const int n = static_cast<int>(ccount[c]);
+          if (n == 0) {                            // that collector is done
+            if (c == 0) cdone0 = true; else cdone1 = true;
+            continue;
+          }
+          const uint32_t* buf = cbuf + 128 * c;
+#pragma unroll
+          for (int r = 0; r < 4; ++r)
+            nx_row[r] = kv_row0 + static_cast<int>(buf[4 * lane + r] & 0x3FFFFFFFu);
+          if (lane < 8) nx_mask = cmask[8 * c + lane];
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_cempty0 + 8u * c);
+          col = c ^ 1;
+          nx_desc = 128u | kDescMasked | kDescGather;
+          return true;
+        }
+        phase = 4;
+      }
+      nx_key0 = it.loc_start + 128 * n_loc++;
+      nx_desc = static_cast<uint32_t>(min(128, it.le - nx_key0)) |
+                (nx_key0 == it.row0 ? kDescCausal : 0u) | (n_loc == it.n_loc_t ? kDescLast : 0u);
+      return true;
+    };
+    for (int t = 0;; ++t) {
+      if (!prepare()) break;
+      const int ks = t % kPairKStages, vs = t % kPairVStages;
+      if (t >= kPairKStages &&
+          !warp_wait(bar_kempty(ks), ((t / kPairKStages) - 1) & 1, wc))
+        break;
+      if (t >= kPairVStages &&
+          !warp_wait(bar_vempty(vs), ((t / kPairVStages) - 1) & 1, wc))
+        break;
+      const uint32_t desc = nx_desc;
+      // publish the tile: its masks, then its descriptor
+      if ((desc & kDescMasked) && lane < 8) tags[vs * 8 + lane] = nx_mask;
+      __syncwarp();
+      if (lane == 0) {
+        tdesc[vs] = desc;
+        mbar_arrive(bar_tag0 + 8u * vs);
+      }
+      const uint32_t kf = bar_kfull(ks), vf = bar_vfull(vs);
+      if (lane == 0) {
+        mbar_arrive_expect_tx(kf, kTileBytes);
+        mbar_arrive_expect_tx(vf, kTileBytes);
+      }
+      __syncwarp();
+      if (desc & kDescGather) {
+        // rows 4 l .. 4 l + 3 of the tile from lane l: one gather4 per operand half
+        const uint32_t roff = lane * 4u * 128u;
+        tma_gather4(s_k(ks) + roff, &tm_kg, kf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
+        tma_gather4(s_k(ks) + kHalfBytes + roff, &tm_kg, kf, 64, nx_row[0], nx_row[1], nx_row[2],
+                    nx_row[3]);
+        tma_gather4(s_v(vs) + roff, &tm_vg, vf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
+        tma_gather4(s_v(vs) + kHalfBytes + roff, &tm_vg, vf, 64, nx_row[0], nx_row[1], nx_row[2],
+                    nx_row[3]);
+      } else if (lane == 0) {
+        tma_load_2d(s_k(ks), &tm_k, kf, 0, kv_row0 + nx_key0);
+        tma_load_2d(s_k(ks) + kHalfBytes, &tm_k, kf, 64, kv_row0 + nx_key0);
+        tma_load_2d(s_v(vs), &tm_v, vf, 0, kv_row0 + nx_key0);
+        tma_load_2d(s_v(vs) + kHalfBytes, &tm_v, vf, 64, kv_row0 + nx_key0);
+      }
+      __syncwarp();
+      issued = t + 1;
+      if (desc & kDescLast) break;
+    }
+    if (lane == 0) {   // no copy may still be in flight when the CTA exits
+      mbar_drain(bar_q, 0, a.wait_ns);
+      for (int t = max(0, issued - kPairKStages); t < issued; ++t)
+        mbar_drain(bar_kfull(t % kPairKStages), (t / kPairKStages) & 1, a.wait_ns);
+      for (int t = max(0, issued - kPairVStages); t < issued; ++t)
+        mbar_drain(bar_vfull(t % kPairVStages), (t / kPairVStages) & 1, a.wait_ns);
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      if (a.debug & 1u) ok = mbar_wait(bar_stall, 0, wc);   // never signalled: test hook
+      if (ok) ok = mbar_wait(bar_q, 0, wc);
+      auto qk = [&](int t, int hd) {
+        const int ks = t % kPairKStages;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32u;
+          mma_bf16_ss(tmem + 128u * hd, smem_desc_sw128(s_q + hd * kTileBytes + off, 16),
+                      smem_desc_sw128(s_k(ks) + off, 16), kIdescQK, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(bar_sfull0 + 8u * hd);
+      };
+      auto pv = [&](int t, int hd) {
+        const int vs = t % kPairVStages;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = smem_desc_sw128(s_v(vs) + kk * 2048u, kHalfBytes);
+          mma_bf16_ts(tmem + 256u + 128u * hd, tmem + 128u * hd + 8u * kk, bd, kIdescPV,
+                      (t > 0 || kk > 0) ? 1u : 0u);
+        }
+      };
+      if (ok) {
+        if ((ok = mbar_wait(bar_kfull(0), 0, wc))) {
+          tc_fence_after();
+          qk(0, 0);
+          qk(0, 1);
+          mma_commit(bar_kempty(0));
+        }
+      }
+      for (int t = 0; ok; ++t) {
+        const int vs = t % kPairVStages;
+        // tile t's descriptor was written before its loads were armed, and
+        // kfull of tile t has been observed (QK(t) is issued)
+        const bool more = a.mode == kModeDense ? t + 1 < it.n_loc_t : (tdesc[vs] & kDescLast) == 0u;
+        // head A: PV(t), then QK(t+1)
+        if (!(ok = mbar_wait(bar_pfull0, t & 1, wc))) break;
+        if (!(ok = mbar_wait(bar_vfull(vs), (t / kPairVStages) & 1, wc))) break;
+        tc_fence_after();
+        pv(t, 0);
+        if (more) {
+          const int ks = (t + 1) % kPairKStages;
+          if (!(ok = mbar_wait(bar_kfull(ks), ((t + 1) / kPairKStages) & 1, wc))) break;
+          tc_fence_after();
+          qk(t + 1, 0);
+        }
+        // head B: PV(t), then QK(t+1)
+        if (!(ok = mbar_wait(bar_pfull0 + 8u, t & 1, wc))) break;
+        tc_fence_after();
+        pv(t, 1);
+        mma_commit(bar_vempty(vs));
+        if (more) {
+          qk(t + 1, 1);
+          mma_commit(bar_kempty((t + 1) % kPairKStages));
+        } else {
+          mma_commit(bar_odone);
+          break;
+        }
+      }
+      mma_commit(bar_drain);
+      mbar_drain(bar_drain, 0, a.wait_ns);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------- collectors (warps 10, 11)
+    // Collector c gathers the keys of the sparse tiles in the bitmap words
+    // w with w % 2 == c into its buffer, 128 at a time, with the tile's
+    // column masks, and hands each buffer to the producer (a count of 0
+    // ends it).
+    const int cpar = warp - 10;
+    const int kt0 = a.sink / 128;
+    const int W = a.tbit_words;
+    const int nw = (pi.n_ct + 31) / 32;
+    // The keys of the tiles that are non-empty and not dense, among the
+    // bitmap words of this collector's parity, taken a window at a time (the
+    // sparse tiles of one bitmap word, lane j holding the j-th), the next
+    // window's masks loaded ahead.
     int sc = 0, swi = -1;
     bool s_done = nw == 0;
     uint32_t sword = 0u;                           // this lane's sparse word of chunk sc
     auto load_sparse_chunk = [&](int c) {
       const int wi = 32 * c + lane;
       sword = 0u;
-      if (wi < nw) sword = (pi.ba[wi] | pi.bb[wi]) & ~(pi.ba[W + wi] | pi.bb[W + wi]);
+      if (wi < nw && (wi & 1) == cpar)
+        sword = (pi.ba[wi] | pi.bb[wi]) & ~(pi.ba[W + wi] | pi.bb[W + wi]);
     };
     bool p_valid = false;                          // prefetched window
     int p_n = 0, p_tile = 0;
@@ -337,237 +557,83 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       scan_next();
     };
     if (nw > 0) {
-      load_dense_chunk(0);
       load_sparse_chunk(0);
       scan_next();
       take_window();
     }
-    int phase = 0;        // 0 sink, 1 dense, 2 gathered, 3 local tiles
-    int n_sink = 0, n_loc = 0;
-    // The next tile, prepared while the previous tile's loads are in flight:
-    // its descriptor, its first key (contiguous tiles), lane l's four rows
-    // 4 l .. 4 l + 3 (gathered tiles) and, in lanes 0-7, word l of the two
-    // heads' column masks (0-3 head A, 4-7 head B).
-    uint32_t nx_desc = 0u;
-    int nx_key0 = 0;
-    int nx_row[4] = {0, 0, 0, 0};
-    uint32_t nx_mask = 0u;
-    auto prepare = [&]() {
-      nx_desc = 0u;
-      if (phase == 0) {
-        if (n_sink < it.n_sink_t) {
-          nx_key0 = 128 * n_sink++;
-          nx_desc = static_cast<uint32_t>(min(128, it.sink_end - nx_key0));
-          return;
-        }
-        phase = 1;
-      }
-      if (phase == 1) {
-        bool full = false;
-        const int j = nw > 0 ? next_dense(full) : -1;
-        if (j >= 0) {
-          if (!full && lane < 8)
-            nx_mask = reinterpret_cast<const uint32_t*>(lane < 4 ? pi.ma + j : pi.mb + j)[lane & 3];
-          nx_key0 = 128 * (kt0 + j);
-          nx_desc = 128u | (full ? 0u : kDescMasked);
-          return;
-        }
-        phase = 2;
-      }
-      if (phase == 2) {
-        // the next 128 keys of the sparse tiles
-        int filled = 0;
-        while (filled < 128 && g_valid) {
-          const int skip = lane == j0 ? cons : 0;
-          const int cnt = lane >= j0 ? g_cnt - skip : 0;
-          int incl = cnt;
+    uint32_t* buf = cbuf + 128 * cpar;
+    for (int n = 0;; ++n) {
+      if (n > 0 && !warp_wait(bar_cempty0 + 8u * cpar, (n - 1) & 1, wc)) break;
+      // the next 128 keys of this collector's sparse tiles
+      int filled = 0;
+      while (filled < 128 && g_valid) {
+        const int skip = lane == j0 ? cons : 0;
+        const int cnt = lane >= j0 ? g_cnt - skip : 0;
+        int incl = cnt;
 #pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(0xffffffffu, incl, o);
-            if (lane >= o) incl += v;
-          }
-          const int excl = incl - cnt;
-          const int tot = __shfl_sync(0xffffffffu, incl, 31);
-          const int take = min(tot, 128 - filled);
-          if (cnt > 0 && excl < take) {
-            // this lane's tile: its keys of rank skip, skip + 1, ... go to
-            // slots filled + excl, ... while they are below filled + take
-            const uint32_t ua[4] = {g_a.x, g_a.y, g_a.z, g_a.w};
-            const uint32_t ub[4] = {g_b.x, g_b.y, g_b.z, g_b.w};
-            const int base_key = 128 * (kt0 + g_tile);
-            int r = 0;
-            for (int w = 0; w < 4; ++w) {
-              uint32_t rem = ua[w] | ub[w];
-              while (rem) {
-                const int bpos = __ffs(rem) - 1;
-                rem &= rem - 1u;
-                if (r >= skip) {
-                  const int pos = excl + r - skip;
-                  if (pos < take)
-                    stage[filled + pos] = static_cast<uint32_t>(base_key + 32 * w + bpos) |
-                                          (((ua[w] >> bpos) & 1u) << 30) |
-                                          (((ub[w] >> bpos) & 1u) << 31);
-                }
-                ++r;
+        for (int o = 1; o < 32; o <<= 1) {
+          const int v = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const int excl = incl - cnt;
+        const int tot = __shfl_sync(0xffffffffu, incl, 31);
+        const int take = min(tot, 128 - filled);
+        if (cnt > 0 && excl < take) {
+          // this lane's tile: its keys of rank skip, skip + 1, ... go to
+          // slots filled + excl, ... while they are below filled + take
+          const uint32_t ua[4] = {g_a.x, g_a.y, g_a.z, g_a.w};
+          const uint32_t ub[4] = {g_b.x, g_b.y, g_b.z, g_b.w};
+          const int base_key = 128 * (kt0 + g_tile);
+          int r = 0;
+          for (int w = 0; w < 4; ++w) {
+            uint32_t rem = ua[w] | ub[w];
+            while (rem) {
+              const int bpos = __ffs(rem) - 1;
+              rem &= rem - 1u;
+              if (r >= skip) {
+                const int pos = excl + r - skip;
+                if (pos < take)
+                  buf[filled + pos] = static_cast<uint32_t>(base_key + 32 * w + bpos) |
+                                        (((ua[w] >> bpos) & 1u) << 30) |
+                                        (((ub[w] >> bpos) & 1u) << 31);
               }
+              ++r;
             }
           }
-          filled += take;
-          if (take == tot) {
-            take_window();
-          } else {
-            // the window continues at the lane holding the first key not taken
-            const uint32_t cut = __ballot_sync(0xffffffffu, cnt > 0 && excl <= take && take < excl + cnt);
-            const int J = __ffs(cut) - 1;
-            const int eJ = __shfl_sync(0xffffffffu, excl, J);
-            cons = (J == j0 ? cons : 0) + (take - eJ);
-            j0 = J;
-          }
         }
-        __syncwarp();
-        if (filled > 0) {
-          const uint32_t first = stage[0] & 0x3FFFFFFFu;
-          for (int r = filled + lane; r < 128; r += 32) stage[r] = first;
-          __syncwarp();
-#pragma unroll
-          for (int r = 0; r < 4; ++r)
-            nx_row[r] = kv_row0 + static_cast<int>(stage[4 * lane + r] & 0x3FFFFFFFu);
-          // column masks: row 32 w + l of the tile is bit l of word w
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const uint32_t e = stage[32 * w + lane];
-            const uint32_t ma = __ballot_sync(0xffffffffu, (e >> 30) & 1u);
-            const uint32_t mb = __ballot_sync(0xffffffffu, (e >> 31) & 1u);
-            if (lane == w) nx_mask = ma;
-            if (lane == 4 + w) nx_mask = mb;
-          }
-          __syncwarp();   // the staging buffer may be refilled for the tile after
-          nx_desc = 128u | kDescMasked | kDescGather;
-          return;
-        }
-        phase = 3;
-      }
-      nx_key0 = it.loc_start + 128 * n_loc++;
-      nx_desc = static_cast<uint32_t>(min(128, it.le - nx_key0)) |
-                (nx_key0 == it.row0 ? kDescCausal : 0u) | (n_loc == it.n_loc_t ? kDescLast : 0u);
-    };
-    prepare();
-    for (int t = 0;; ++t) {
-      const int ks = t % kPairKStages, vs = t % kPairVStages;
-      if (t >= kPairKStages &&
-          !warp_wait(bar_kempty(ks), ((t / kPairKStages) - 1) & 1, wc))
-        break;
-      if (t >= kPairVStages &&
-          !warp_wait(bar_vempty(vs), ((t / kPairVStages) - 1) & 1, wc))
-        break;
-      const uint32_t desc = nx_desc;
-      // publish the tile: its masks, then its descriptor
-      if ((desc & kDescMasked) && lane < 8) tags[vs * 8 + lane] = nx_mask;
-      __syncwarp();
-      if (lane == 0) {
-        tdesc[vs] = desc;
-        mbar_arrive(bar_tag0 + 8u * vs);
-      }
-      const uint32_t kf = bar_kfull(ks), vf = bar_vfull(vs);
-      if (lane == 0) {
-        mbar_arrive_expect_tx(kf, kTileBytes);
-        mbar_arrive_expect_tx(vf, kTileBytes);
-      }
-      __syncwarp();
-      if (desc & kDescGather) {
-        // rows 4 l .. 4 l + 3 of the tile from lane l: one gather4 per operand half
-        const uint32_t roff = lane * 4u * 128u;
-        tma_gather4(s_k(ks) + roff, &tm_kg, kf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
-        tma_gather4(s_k(ks) + kHalfBytes + roff, &tm_kg, kf, 64, nx_row[0], nx_row[1], nx_row[2],
-                    nx_row[3]);
-        tma_gather4(s_v(vs) + roff, &tm_vg, vf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
-        tma_gather4(s_v(vs) + kHalfBytes + roff, &tm_vg, vf, 64, nx_row[0], nx_row[1], nx_row[2],
-                    nx_row[3]);
-      } else if (lane == 0) {
-        tma_load_2d(s_k(ks), &tm_k, kf, 0, kv_row0 + nx_key0);
-        tma_load_2d(s_k(ks) + kHalfBytes, &tm_k, kf, 64, kv_row0 + nx_key0);
-        tma_load_2d(s_v(vs), &tm_v, vf, 0, kv_row0 + nx_key0);
-        tma_load_2d(s_v(vs) + kHalfBytes, &tm_v, vf, 64, kv_row0 + nx_key0);
-      }
-      __syncwarp();
-      issued = t + 1;
-      if (desc & kDescLast) break;
-      prepare();
-    }
-    if (lane == 0) {   // no copy may still be in flight when the CTA exits
-      mbar_drain(bar_q, 0, a.wait_ns);
-      for (int t = max(0, issued - kPairKStages); t < issued; ++t)
-        mbar_drain(bar_kfull(t % kPairKStages), (t / kPairKStages) & 1, a.wait_ns);
-      for (int t = max(0, issued - kPairVStages); t < issued; ++t)
-        mbar_drain(bar_vfull(t % kPairVStages), (t / kPairVStages) & 1, a.wait_ns);
-    }
-  } else if (warp == 9) {
-    // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = true;
-      if (a.debug & 1u) ok = mbar_wait(bar_stall, 0, wc);   // never signalled: test hook
-      if (ok) ok = mbar_wait(bar_q, 0, wc);
-      auto qk = [&](int t, int hd) {
-        const int ks = t % kPairKStages;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalfBytes + (kk & 3) * 32u;
-          mma_bf16_ss(tmem + 128u * hd, smem_desc_sw128(s_q + hd * kTileBytes + off, 16),
-                      smem_desc_sw128(s_k(ks) + off, 16), kIdescQK, kk > 0 ? 1u : 0u);
-        }
-        mma_commit(bar_sfull0 + 8u * hd);
-      };
-      auto pv = [&](int t, int hd) {
-        const int vs = t % kPairVStages;
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint64_t bd = smem_desc_sw128(s_v(vs) + kk * 2048u, kHalfBytes);
-          mma_bf16_ts(tmem + 256u + 128u * hd, tmem + 128u * hd + 8u * kk, bd, kIdescPV,
-                      (t > 0 || kk > 0) ? 1u : 0u);
-        }
-      };
-      if (ok) {
-        if ((ok = mbar_wait(bar_kfull(0), 0, wc))) {
-          tc_fence_after();
-          qk(0, 0);
-          qk(0, 1);
-          mma_commit(bar_kempty(0));
-        }
-      }
-      for (int t = 0; ok; ++t) {
-        const int vs = t % kPairVStages;
-        // tile t's descriptor was written before its loads were armed, and
-        // kfull of tile t has been observed (QK(t) is issued)
-        const bool more = (tdesc[vs] & kDescLast) == 0u;
-        // head A: PV(t), then QK(t+1)
-        if (!(ok = mbar_wait(bar_pfull0, t & 1, wc))) break;
-        if (!(ok = mbar_wait(bar_vfull(vs), (t / kPairVStages) & 1, wc))) break;
-        tc_fence_after();
-        pv(t, 0);
-        if (more) {
-          const int ks = (t + 1) % kPairKStages;
-          if (!(ok = mbar_wait(bar_kfull(ks), ((t + 1) / kPairKStages) & 1, wc))) break;
-          tc_fence_after();
-          qk(t + 1, 0);
-        }
-        // head B: PV(t), then QK(t+1)
-        if (!(ok = mbar_wait(bar_pfull0 + 8u, t & 1, wc))) break;
-        tc_fence_after();
-        pv(t, 1);
-        mma_commit(bar_vempty(vs));
-        if (more) {
-          qk(t + 1, 1);
-          mma_commit(bar_kempty((t + 1) % kPairKStages));
+        filled += take;
+        if (take == tot) {
+          take_window();
         } else {
-          mma_commit(bar_odone);
-          break;
+          // the window continues at the lane holding the first key not taken
+          const uint32_t cut = __ballot_sync(0xffffffffu, cnt > 0 && excl <= take && take < excl + cnt);
+          const int J = __ffs(cut) - 1;
+          const int eJ = __shfl_sync(0xffffffffu, excl, J);
+          cons = (J == j0 ? cons : 0) + (take - eJ);
+          j0 = J;
         }
       }
-      mma_commit(bar_drain);
-      mbar_drain(bar_drain, 0, a.wait_ns);
+      __syncwarp();
+      if (filled > 0) {
+        const uint32_t first = buf[0] & 0x3FFFFFFFu;
+        for (int r = filled + lane; r < 128; r += 32) buf[r] = first;
+        __syncwarp();
+        // column masks: row 32 w + l of the tile is bit l of word w
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const uint32_t e = buf[32 * w + lane];
+          const uint32_t ma = __ballot_sync(0xffffffffu, (e >> 30) & 1u);
+          const uint32_t mb = __ballot_sync(0xffffffffu, (e >> 31) & 1u);
+          if (lane == w) cmask[8 * cpar + w] = ma;
+          if (lane == 4 + w) cmask[8 * cpar + 4 + w] = mb;
+        }
+      }
+      if (lane == 0) ccount[cpar] = static_cast<uint32_t>(filled);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_cfull0 + 8u * cpar);
+      if (filled == 0) break;
     }
-    __syncwarp();
-  }   // warps 10-11 have no role
+  }
   } else {
     // ------------------------------------------------------------- softmax
     asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
@@ -584,17 +650,18 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     for (int t = 0; !last; ++t) {
       if (!(ok = warp_wait(bar_sfull0 + 8u * hd, t & 1, wc))) break;
       tc_fence_after();
-      uint32_t sr[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + s_col + 32u * c, sr[c]);
-      // while S comes out of TMEM: the tile's descriptor and masks (every
-      // tile arrives once on its V slot's tag barrier, before its loads)
       const int vs = t % kPairVStages;
-      if (!(ok = warp_wait(bar_tag0 + 8u * vs, (t / kPairVStages) & 1, wc))) {
-        tmem_ld_wait();
-        break;
+      uint32_t dw;
+      if (a.mode == kModeDense) {
+        // every tile is a local tile from key 0: its descriptor is known here
+        const int k0 = 128 * t;
+        dw = static_cast<uint32_t>(min(128, it.le - k0)) | (k0 == it.row0 ? kDescCausal : 0u) |
+             (t + 1 == it.n_loc_t ? kDescLast : 0u);
+      } else {
+        // every tile arrives once on its V slot's tag barrier, before its loads
+        if (!(ok = warp_wait(bar_tag0 + 8u * vs, (t / kPairVStages) & 1, wc))) break;
+        dw = tdesc[vs];
       }
-      const uint32_t dw = tdesc[vs];
       last = (dw & kDescLast) != 0u;
       const int valid = static_cast<int>(dw & 0x1FFu);
       const int limit = (dw & kDescCausal) ? min(valid, r + 1) : valid;
@@ -603,18 +670,19 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
         for (int w = 0; w < 4; ++w) tw[w] = tags[(vs * 2 + hd) * 4 + w];
       }
-      tmem_ld_wait();
-      // mask the 32-key words with a missing key or past the limit (the head
-      // masks are the same for the whole warp)
+      uint32_t sr[4][32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        if (c * 32 + 31 >= limit || tw[c] != 0xffffffffu) {
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + s_col + 32u * c, sr[c]);
+      tmem_ld_wait();
+      const bool masked = (limit < 128) || ((tw[0] & tw[1] & tw[2] & tw[3]) != 0xffffffffu);
+      if (masked) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const bool v = (c * 32 + e < limit) && ((tw[c] >> e) & 1u);
             if (!v) sr[c][e] = __float_as_uint(-INFINITY);
           }
-        }
       }
       float mxv[8];
 #pragma unroll
