@@ -402,7 +402,9 @@ def sweep():
             ts.append(a.elapsed_time(b))
         return statistics.median(ts)
 
-    plan = [(C4_SWEEP_128K, THETA_DENSITY_SWEEP), (C4_B4_16K, THETA_DENSITY_SWEEP),
+    # theta = -inf keeps only the sink and local keys: the attention time of
+    # that point is what the sink and local tiles cost inside every step
+    plan = [(C4_SWEEP_128K, THETA_DENSITY_SWEEP + (-math.inf,)), (C4_B4_16K, THETA_DENSITY_SWEEP),
             (C3_QWEN_64K, (5.0,))]
     for w, thetas in plan:
         inp = generate(w)

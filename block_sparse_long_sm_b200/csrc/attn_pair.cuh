@@ -498,17 +498,29 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     const int W = a.tbit_words;
     const int nw = (pi.n_ct + 31) / 32;
     // The keys of the tiles that are non-empty and not dense, among the
-    // bitmap words of this collector's parity, taken a window at a time (the
-    // sparse tiles of one bitmap word, lane j holding the j-th), the next
-    // window's masks loaded ahead.
-    int sc = 0, swi = -1;
+    // bitmap words of this collector's parity, taken a window of 32 such
+    // tiles at a time (lane j holding the j-th), the next window's masks
+    // loaded ahead.  The bitmap is read 32 words (1024 tiles) at a time.
+    int sc = 0;
     bool s_done = nw == 0;
     uint32_t sword = 0u;                           // this lane's sparse word of chunk sc
+    int sbase = 0;                                 // rank of its first sparse tile in the chunk
+    int stot = 0, srank = 0;                       // sparse tiles in the chunk, handed out
     auto load_sparse_chunk = [&](int c) {
       const int wi = 32 * c + lane;
       sword = 0u;
       if (wi < nw && (wi & 1) == cpar)
         sword = (pi.ba[wi] | pi.bb[wi]) & ~(pi.ba[W + wi] | pi.bb[W + wi]);
+      const int cw = __popc(sword);
+      int incl = cw;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += v;
+      }
+      sbase = incl - cw;
+      stot = __shfl_sync(0xffffffffu, incl, 31);
+      srank = 0;
     };
     bool p_valid = false;                          // prefetched window
     int p_n = 0, p_tile = 0;
@@ -516,22 +528,30 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     auto scan_next = [&]() {
       p_valid = false;
       while (!s_done) {
-        const uint32_t cand = __ballot_sync(0xffffffffu, sword != 0u) &
-                              (swi < 31 ? (0xffffffffu << (swi + 1)) : 0u);
-        if (cand) {
-          swi = __ffs(cand) - 1;
-          const uint32_t word = __shfl_sync(0xffffffffu, sword, swi);
-          p_n = __popc(word);
+        if (srank < stot) {
+          // lane j: the sparse tile of rank srank + j, in the last word whose
+          // first rank is at most that
+          const int R = srank + lane;
+          int w = 0;
+#pragma unroll
+          for (int step = 16; step > 0; step >>= 1) {
+            const int c = w + step;
+            const int bc = __shfl_sync(0xffffffffu, sbase, c & 31);
+            if (c < 32 && bc <= R) w = c;
+          }
+          const uint32_t word = __shfl_sync(0xffffffffu, sword, w);
+          const int wb = __shfl_sync(0xffffffffu, sbase, w);
+          p_n = min(32, stot - srank);
           if (lane < p_n) {
-            p_tile = 32 * (32 * sc + swi) + static_cast<int>(__fns(word, 0, lane + 1));
+            p_tile = 32 * (32 * sc + w) + static_cast<int>(__fns(word, 0, R - wb + 1));
             p_a = pi.ma[p_tile];
             p_b = pi.mb[p_tile];
           }
+          srank += p_n;
           p_valid = true;
           return;
         }
         ++sc;
-        swi = -1;
         if (32 * sc >= nw) {
           s_done = true;
           return;
@@ -647,16 +667,41 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     float lsum = 0.f;
     bool ok = true;
     bool last = false;
+    // When both heads keep every key of every candidate tile (the near-dense
+    // case), the tiles are sink, n_ct full tiles and local, in the producer's
+    // order, and their descriptors are known here without waiting for them.
+    bool known = a.mode == kModeDense;
+    if (!known && pi.n_ct > 0) {
+      const int nwf = (pi.n_ct + 31) / 32;
+      int missing = 0;
+      for (int w0 = 0; w0 < nwf; w0 += 32) {
+        const int wi = w0 + lane;
+        if (wi < nwf) {
+          const uint32_t f = pi.ba[2 * a.tbit_words + wi] & pi.bb[2 * a.tbit_words + wi];
+          const int n = min(32, pi.n_ct - 32 * wi);
+          const uint32_t need = n >= 32 ? 0xffffffffu : ((1u << n) - 1u);
+          missing += (f & need) != need ? 1 : 0;
+        }
+      }
+      known = __reduce_add_sync(0xffffffffu, missing) == 0;
+    }
+    const int n_full = a.mode == kModeDense ? 0 : pi.n_ct;
     for (int t = 0; !last; ++t) {
       if (!(ok = warp_wait(bar_sfull0 + 8u * hd, t & 1, wc))) break;
       tc_fence_after();
       const int vs = t % kPairVStages;
       uint32_t dw;
-      if (a.mode == kModeDense) {
-        // every tile is a local tile from key 0: its descriptor is known here
-        const int k0 = 128 * t;
-        dw = static_cast<uint32_t>(min(128, it.le - k0)) | (k0 == it.row0 ? kDescCausal : 0u) |
-             (t + 1 == it.n_loc_t ? kDescLast : 0u);
+      if (known) {
+        if (t < it.n_sink_t) {
+          dw = static_cast<uint32_t>(min(128, it.sink_end - 128 * t));
+        } else if (t < it.n_sink_t + n_full) {
+          dw = 128u;
+        } else {
+          const int li = t - it.n_sink_t - n_full;
+          const int k0 = it.loc_start + 128 * li;
+          dw = static_cast<uint32_t>(min(128, it.le - k0)) | (k0 == it.row0 ? kDescCausal : 0u) |
+               (li + 1 == it.n_loc_t ? kDescLast : 0u);
+        }
       } else {
         // every tile arrives once on its V slot's tag barrier, before its loads
         if (!(ok = warp_wait(bar_tag0 + 8u * vs, (t / kPairVStages) & 1, wc))) break;

@@ -99,6 +99,8 @@ constexpr int kSaleThreads = 320;            // warp 0 TMA, warp 1 MMA, warps 2-
 constexpr int kSaleStages = 8;
 constexpr int kSaleKeys = 64;                // keys per K tile
 constexpr int kSaleHeads = 4;                // q heads per CTA
+constexpr int kSaleBufs = 2;                 // accumulator sets in TMEM (kSaleBufs * kSaleHeads * 64 <= 512)
+static_assert(kSaleBufs * kSaleHeads * 64 <= 512, "more TMEM columns than a CTA has");
 constexpr uint32_t kQ8Bytes = 128u * 128u;   // 128 rows x 128 int8
 constexpr uint32_t kK8Bytes = kSaleKeys * 128u;
 constexpr int kMaxGroupWords = 512;          // candidate 16-key groups / 32 (L <= 262144)
@@ -138,8 +140,8 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
   auto bar_full = [&](int st) { return b0 + 8u * (1 + st); };
   auto bar_empty = [&](int st) { return b0 + 8u * (1 + kSaleStages + st); };
   auto bar_afull = [&](int bb) { return b0 + 8u * (1 + 2 * kSaleStages + bb); };
-  auto bar_afree = [&](int bb) { return b0 + 8u * (3 + 2 * kSaleStages + bb); };
-  const uint32_t bar_drain = b0 + 8u * (5 + 2 * kSaleStages);
+  auto bar_afree = [&](int bb) { return b0 + 8u * (1 + 2 * kSaleStages + kSaleBufs + bb); };
+  const uint32_t bar_drain = b0 + 8u * (1 + 2 * kSaleStages + 2 * kSaleBufs);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 512);
   volatile uint32_t* abort_flag = tmem_holder + 1;
   uint32_t* gflags = reinterpret_cast<uint32_t*>(bar_area + 1024);       // [head][words]
@@ -176,9 +178,9 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
       mbar_init(bar_full(st), 1);
       mbar_init(bar_empty(st), 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kSaleBufs; ++i) {
       mbar_init(bar_afull(i), 1);
-      mbar_init(bar_afree(i), 256);
+      mbar_init(bar_afree(i), 8);                  // the eight epilogue warps
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0u;
@@ -224,9 +226,9 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
     if (lane == 0) {
       bool ok = mbar_wait(bar_q, 0, wc);
       for (int t = 0; ok && t < T; ++t) {
-        const int st = t % kSaleStages, bb = t & 1;
+        const int st = t % kSaleStages, bb = t % kSaleBufs;
         if (!(ok = mbar_wait(bar_full(st), (t / kSaleStages) & 1, wc))) break;
-        if (t >= 2 && !(ok = mbar_wait(bar_afree(bb), ((t >> 1) - 1) & 1, wc))) break;
+        if (t >= kSaleBufs && !(ok = mbar_wait(bar_afree(bb), ((t / kSaleBufs) - 1) & 1, wc))) break;
         tc_fence_after();
         for (int j = 0; j < nh; ++j) {
 #pragma unroll
@@ -260,17 +262,16 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
       thr[u] = INFINITY;
     }
     for (int t = 0; t < T; ++t) {
-      const int bb = t & 1;
-      if (!warp_wait(bar_afull(bb), (t >> 1) & 1, wc)) break;
+      const int bb = t % kSaleBufs;
+      if (!warp_wait(bar_afull(bb), (t / kSaleBufs) & 1, wc)) break;
       tc_fence_after();
       const int key0 = tile_key0(t);
-      uint32_t gbits = 0;                              // bit 4u + g: head hsel + 2u, group g
+      if (t < n_stat_t) {
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int j = hsel + 2 * u;
-        if (j >= nh) continue;                         // warp-uniform
-        const uint32_t taddr = tmem + lane_off + 64u * (bb * kSaleHeads + j);
-        if (t < n_stat_t) {
+        for (int u = 0; u < 2; ++u) {
+          const int j = hsel + 2 * u;
+          if (j >= nh) continue;                       // warp-uniform
+          const uint32_t taddr = tmem + lane_off + 64u * (bb * kSaleHeads + j);
           uint32_t sr[2][32];
           tmem_ld32(taddr, sr[0]);
           tmem_ld32(taddr + 32u, sr[1]);
@@ -305,39 +306,49 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
           if (t == n_stat_t - 1)
             thr[u] = row_valid ? m[u] + logf(a.tau_h[h0 + hsel + 2 * u] * l[u])   // t_i = em + ln(tau el)
                                : INFINITY;
-        } else {
-          uint32_t pk[32];
-          tmem_ld32_pack16(taddr, pk);
-          tmem_ld_wait();
+        }
+      } else {
+        // both heads' 64 columns as packed 16-bit pairs, one wait for the two
+        // loads; the four 16-key groups' K scales are read meanwhile
+        uint32_t pk[2][32];
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {               // 16 keys = 8 packed registers
-            const uint32_t* q = pk + 8 * g;
+        for (int u = 0; u < 2; ++u)
+          if (hsel + 2 * u < nh) tmem_ld32_pack16(tmem + lane_off + 64u * (bb * kSaleHeads + hsel + 2 * u), pk[u]);
+        float ksg[4];
+#pragma unroll
+        for (int g = 0; g < 4; ++g) ksg[g] = kscale[min(key0 + 16 * g, cand_hi - 1) >> a.bk_log2];
+        tmem_ld_wait();
+        uint32_t gbits = 0;                            // bit 4u + g: head hsel + 2u, group g
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          if (hsel + 2 * u >= nh) continue;            // warp-uniform
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {                // 16 keys = 8 packed registers
+            const uint32_t* q = pk[u] + 8 * g;
             const uint32_t m01 = max_s16x2(max_s16x2(q[0], q[1]), max_s16x2(q[2], q[3]));
             const uint32_t m23 = max_s16x2(max_s16x2(q[4], q[5]), max_s16x2(q[6], q[7]));
             const uint32_t mm = max_s16x2(m01, m23);
             const int mx = max(static_cast<int>(static_cast<int16_t>(mm & 0xffffu)),
                                static_cast<int>(mm) >> 16);
-            const int key = key0 + 16 * g;
-            if (key < cand_hi && static_cast<float>(mx) * (cq[u] * kscale[key >> a.bk_log2]) >= thr[u])
+            if (key0 + 16 * g < cand_hi && static_cast<float>(mx) * (cq[u] * ksg[g]) >= thr[u])
               gbits |= 1u << (4 * u + g);
           }
         }
-      }
-      if (t >= n_stat_t) {
         // one warp reduction and at most two shared atomics per tile for both heads
         gbits = __reduce_or_sync(0xffffffffu, gbits);
         if (lane == 0 && gbits) {
-          const int g0 = (key0 - cand_lo) / 16;      // multiple of 4: one word holds 4 bits
+          const int g0 = (key0 - cand_lo) / 16;        // multiple of 4: one word holds 4 bits
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const uint32_t bits = (gbits >> (4 * u)) & 0xfu;
             if (bits) atomicOr(&gflags[(hsel + 2 * u) * kMaxGroupWords + (g0 >> 5)], bits << (g0 & 31));
           }
         }
-        gbits = 0;
       }
+      // the buffer is free once every epilogue warp has read it: one arrival per warp
       tc_fence_before();
-      mbar_arrive(bar_afree(bb));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_afree(bb));
     }
   }
   tc_fence_before();

@@ -161,3 +161,42 @@ def test_step_grouping(step, hq, hkv):
     compare_anchor_masks(run, inp, heads)
     rows = {hd: sample_rows(L, 30, 5 * hd[1] + step, must=(L - 1, 2047, 2048)) for hd in heads}
     compare_outputs(run, inp, rows)
+
+
+def test_c4_sweep_128k_operating_points():
+    """The density sweep's layer at full size (its own seed), at the sweep's
+    thresholds between the near-dense and the sparse ends: sampled blocks of
+    three heads bit-exact up to near-ties, sampled rows within the stated
+    bound, in the launch configuration the benchmark times."""
+    from workloads import C4_SWEEP_128K
+    w = C4_SWEEP_128K
+    inp = generate(w)
+    dev = None
+    heads = [(0, 0), (0, 13), (0, 30)]
+    for theta in (7.0, 4.0, 2.5, 2.0):
+        run = Run(inp, mode="anchor", sink=w.sink, local=w.local, theta=theta, dev=dev)
+        dev = (run.q, run.k, run.v)
+        compare_anchor_masks(run, inp, heads,
+                             blocks_of=lambda b, h: edge_blocks(w.seq_len, 3, h + int(theta)))
+        rows = {hd: sample_rows(w.seq_len, 10, hd[1] + int(10 * theta), must=(w.seq_len - 1,))
+                for hd in heads}
+        compare_outputs(run, inp, rows)
+        del run
+
+
+def test_c4_sweep_128k_theta_inf_equals_dense_mode():
+    from workloads import C4_SWEEP_128K
+    w = C4_SWEEP_128K
+    inp = generate(w, kv_groups=[0, 7])
+    run_inf = Run(inp, mode="anchor", sink=w.sink, local=w.local, theta=math.inf)
+    assert run_inf.stats.kept_pairs == run_inf.stats.dense_pairs
+    rows = {(0, h): sample_rows(w.seq_len, 10, h, must=(0, w.seq_len - 1)) for h in (0, 3, 29)}
+    compare_outputs(run_inf, inp, rows, dense=True)
+    o_inf = run_inf.o.clone()
+    run_dense = Run(inp, mode="dense", sink=w.sink, local=w.local,
+                    dev=(run_inf.q, run_inf.k, run_inf.v))
+    compare_outputs(run_dense, inp, rows, dense=True)
+    # the same key sets through the two tile paths (candidate tiles vs
+    # contiguous local tiles): outputs within bf16 rounding of each other
+    d = (o_inf.float() - run_dense.o.float()).abs()
+    assert float(d.max()) <= 2 * 2.0 ** -8 * float(run_dense.o.float().abs().max()) + 1e-3

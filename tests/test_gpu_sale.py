@@ -87,3 +87,17 @@ def test_sale_strong_sink_local128(hq, tau):
     compare_outputs(run, inp, {hd: range(L) for hd in heads}, bound="bf16")
     dense = Run(inp, mode="dense", sink=sink, local=local)
     compare_outputs(dense, inp, {hd: range(L) for hd in heads}, dense=True, bound="bf16")
+
+
+def test_sale_c2_full_size_pruning_tau():
+    """SALE on the 128K layer at a threshold that skips key blocks (tau =
+    0.1 keeps about 45 % of the candidate blocks on these inputs): sampled
+    blocks bit-exact up to near-ties, sampled rows within the stated bound."""
+    w = C2_LLAMA_128K
+    inp = generate(w, kv_groups=[0, 7])
+    run = Run(inp, mode="sale", sink=w.sink, local=w.local, tau=0.1, block_k=w.block_k)
+    assert run.stats.kept_candidates < 0.8 * run.stats.candidates, "the case must prune"
+    heads = [(0, 0), (0, 3), (0, 30)]
+    compare_sale_masks(run, inp, heads, blocks_of=lambda b, h: edge_blocks(w.seq_len, 3, h))
+    rows = {hd: sample_rows(w.seq_len, 10, hd[1], must=(w.seq_len - 1,)) for hd in heads}
+    compare_outputs(run, inp, rows)
