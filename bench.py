@@ -741,8 +741,8 @@ def variant_bench(args, w: Workload):
 
 
 # SALE thresholds that really skip key blocks on the synthetic 128K layer
-# (the oracle keeps about 46 % of the candidate blocks at 0.1)
-SALE_PRUNING_TAUS = (0.1,)
+# (about 45 % of the candidate blocks kept at 0.1, about 10 % at 0.3)
+SALE_PRUNING_TAUS = (0.1, 0.3)
 
 
 def _operating_point(spa, torch, timed, p, ws, q, k, v, o, stream, peaks, dense_ms, label):

@@ -3,8 +3,8 @@
 Usage: ``python -m block_sparse_long_sm_b200.build [--force]`` (or
 ``build()`` from Python).  The build is incremental: it is skipped when the
 library is newer than every source under ``csrc/`` and ``include/``.  Extra
-nvcc flags (for example ``-DSPA_EXP2_POLY_EVERY=4``) can be passed through
-the ``SPA_NVCC_EXTRA`` environment variable together with ``--force``.
+nvcc flags (for example ``-Xptxas -v``) can be passed through the
+``SPA_NVCC_EXTRA`` environment variable together with ``--force``.
 """
 
 from __future__ import annotations

@@ -151,7 +151,9 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
                         const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_kg,
                         const __grid_constant__ CUtensorMap tm_v,
-                        const __grid_constant__ CUtensorMap tm_vg, const AttnArgs a) {
+                        const __grid_constant__ CUtensorMap tm_vg,
+                        const __grid_constant__ CUtensorMap tm_k16,
+                        const __grid_constant__ CUtensorMap tm_v16, const AttnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -228,6 +230,8 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
     prefetch_tensormap(&tm_kg);
     prefetch_tensormap(&tm_v);
     prefetch_tensormap(&tm_vg);
+    prefetch_tensormap(&tm_k16);
+    prefetch_tensormap(&tm_v16);
   }
   tc_fence_before();
   __syncthreads();
@@ -396,14 +400,28 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
       }
       __syncwarp();
       if (desc & kDescGather) {
-        // rows 4 l .. 4 l + 3 of the tile from lane l: one gather4 per operand half
+        // rows 4 l .. 4 l + 3 of the tile from lane l: one gather4 per operand
+        // half; a 16-row chunk (lanes 4 c .. 4 c + 3) of consecutive keys, as
+        // every chunk of a selection in 16-key blocks is, is one tiled box
+        // per operand half from its first lane instead
         const uint32_t roff = lane * 4u * 128u;
-        tma_gather4(s_k(ks) + roff, &tm_kg, kf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
-        tma_gather4(s_k(ks) + kHalfBytes + roff, &tm_kg, kf, 64, nx_row[0], nx_row[1], nx_row[2],
-                    nx_row[3]);
-        tma_gather4(s_v(vs) + roff, &tm_vg, vf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
-        tma_gather4(s_v(vs) + kHalfBytes + roff, &tm_vg, vf, 64, nx_row[0], nx_row[1], nx_row[2],
-                    nx_row[3]);
+        const int prev_last = __shfl_up_sync(0xffffffffu, nx_row[3], 1);
+        const bool seq = nx_row[1] == nx_row[0] + 1 && nx_row[2] == nx_row[0] + 2 &&
+                         nx_row[3] == nx_row[0] + 3 && ((lane & 3) == 0 || prev_last + 1 == nx_row[0]);
+        const uint32_t seq_bits = __ballot_sync(0xffffffffu, seq);
+        if (((seq_bits >> (lane & ~3)) & 0xFu) != 0xFu) {
+          tma_gather4(s_k(ks) + roff, &tm_kg, kf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
+          tma_gather4(s_k(ks) + kHalfBytes + roff, &tm_kg, kf, 64, nx_row[0], nx_row[1], nx_row[2],
+                      nx_row[3]);
+          tma_gather4(s_v(vs) + roff, &tm_vg, vf, 0, nx_row[0], nx_row[1], nx_row[2], nx_row[3]);
+          tma_gather4(s_v(vs) + kHalfBytes + roff, &tm_vg, vf, 64, nx_row[0], nx_row[1], nx_row[2],
+                      nx_row[3]);
+        } else if ((lane & 3) == 0) {
+          tma_load_2d(s_k(ks) + roff, &tm_k16, kf, 0, nx_row[0]);
+          tma_load_2d(s_k(ks) + kHalfBytes + roff, &tm_k16, kf, 64, nx_row[0]);
+          tma_load_2d(s_v(vs) + roff, &tm_v16, vf, 0, nx_row[0]);
+          tma_load_2d(s_v(vs) + kHalfBytes + roff, &tm_v16, vf, 64, nx_row[0]);
+        }
       } else if (lane == 0) {
         tma_load_2d(s_k(ks), &tm_k, kf, 0, kv_row0 + nx_key0);
         tma_load_2d(s_k(ks) + kHalfBytes, &tm_k, kf, 64, kv_row0 + nx_key0);
@@ -598,7 +616,33 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
         const int excl = incl - cnt;
         const int tot = __shfl_sync(0xffffffffu, incl, 31);
         const int take = min(tot, 128 - filled);
-        if (cnt > 0 && excl < take) {
+        const bool mine = cnt > 0 && excl < take;
+        const uint32_t act = __ballot_sync(0xffffffffu, mine);
+        if (__reduce_max_sync(0xffffffffu, mine ? g_cnt : 0) > 6 * __popc(act)) {
+          // few tiles with many keys each (a bit loop per lane would be
+          // long): the warp places one tile's keys at a time, a 32-key word
+          // per step, lane l taking column l
+          for (uint32_t rest = act; rest; rest &= rest - 1u) {
+            const int j = __ffs(rest) - 1;
+            const int ex = __shfl_sync(0xffffffffu, excl, j);
+            const int sk = __shfl_sync(0xffffffffu, skip, j);
+            const int base_key = 128 * (kt0 + __shfl_sync(0xffffffffu, g_tile, j));
+            int rbase = 0;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              // word w of lane j's two masks (each lane passes its own word w)
+              const uint32_t ua = __shfl_sync(0xffffffffu, w == 0 ? g_a.x : w == 1 ? g_a.y : w == 2 ? g_a.z : g_a.w, j);
+              const uint32_t ub = __shfl_sync(0xffffffffu, w == 0 ? g_b.x : w == 1 ? g_b.y : w == 2 ? g_b.z : g_b.w, j);
+              const uint32_t m = ua | ub;
+              const int rk = rbase + __popc(m & ((1u << lane) - 1u));
+              const int pos = ex + rk - sk;
+              if (((m >> lane) & 1u) && rk >= sk && pos < take)
+                buf[filled + pos] = static_cast<uint32_t>(base_key + 32 * w + lane) |
+                                    (((ua >> lane) & 1u) << 30) | (((ub >> lane) & 1u) << 31);
+              rbase += __popc(m);
+            }
+          }
+        } else if (mine) {
           // this lane's tile: its keys of rank skip, skip + 1, ... go to
           // slots filled + excl, ... while they are below filled + take
           const uint32_t ua[4] = {g_a.x, g_a.y, g_a.z, g_a.w};

@@ -548,14 +548,14 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 // words as its tile mask.  Stores, by density of the warp's 32 words: all
 // keys kept -- one shuffle and one coalesced store of the same 32 values per
 // row; at most 8 keys in every word -- each thread stores its own row's keys;
-// in between -- the rows' (word, list position) pairs are staged and each row
-// with keys is one coalesced store.  CTAs are numbered heaviest first (last M
+// in between -- row by row, the row's word and list position shuffled to the
+// warp, one coalesced store of its kept keys.  CTAs are numbered heaviest first (last M
 // tile first), so the block scheduler fills the GPU longest-job-first.
 constexpr int kSelEpiWarps = 16;
 constexpr int kSelThreads = 32 * (2 + kSelEpiWarps);
 constexpr int kSelStages = 4;
 constexpr int kSelBufs = 4;
-constexpr uint32_t kSelBarBytes = 16384u;   // barriers, TMEM slot, word exchange, store staging
+constexpr uint32_t kSelBarBytes = 8192u;    // barriers, TMEM slot, word exchange
 constexpr uint32_t kSelSmemBytes = 1024u + 2u * kTileBytes + kSelStages * kTileBytes + kSelBarBytes;
 static_assert(kSelSmemBytes <= 232448u, "more shared memory than a CTA may use");
 
@@ -602,7 +602,6 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_area + 256);
   volatile uint32_t* abort_flag = tmem_holder + 1;
   uint4* x_words = reinterpret_cast<uint4*>(bar_area + 1024);     // [2][128 rows]: 4 words
-  uint4* stage = reinterpret_cast<uint4*>(bar_area + 5120);       // [16 warps][32 rows], 8 KB
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // item: heaviest M tile first
@@ -636,10 +635,10 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
     }
     for (int i = 0; i < kSelBufs; ++i) {
       mbar_init(bar_sfull(i), 1);
-      mbar_init(bar_sfree(i), 32 * kSelEpiWarps);
+      mbar_init(bar_sfree(i), kSelEpiWarps);       // one arrival per epilogue warp
     }
-    mbar_init(bar_x(0), 32 * kSelEpiWarps);
-    mbar_init(bar_x(1), 32 * kSelEpiWarps);
+    mbar_init(bar_x(0), kSelEpiWarps);
+    mbar_init(bar_x(1), kSelEpiWarps);
     mbar_init(bar_drain, 1);
     *abort_flag = 0u;
     fence_barrier_init();
@@ -721,7 +720,6 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
     uint32_t* row_bits = a.tbits + ((long long)bh * a.nqb + qb) * 3 * a.tbit_words;
     uint32_t occ_acc = 0u, den_acc = 0u, full_acc = 0u;   // this row's tile bits, 32 tiles at a time
     const uint32_t lt = (1u << lane) - 1u;
-    uint4* my_stage = stage + (warp - 2) * 32;
     const uint32_t below_q = (1u << qtr) - 1u;  // words of this row before this warp's
     for (int t = 0; t < T; ++t) {
       const int bb = t % kSelBufs, xs = t & 1;
@@ -731,7 +729,8 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
       tmem_ld32(tmem + lane_off + 128u * bb + 32u * qtr, sr);
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(bar_sfree(bb));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_sfree(bb));
       const int key0 = (kt0 + t) * 128 + 32 * qtr;
       // candidate keys of this row inside these 32 columns: [lo, hi)
       const int lo = max(a.sink - key0, 0);
@@ -749,7 +748,8 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
       for (int o = 1; o < a.step; o <<= 1) w |= __shfl_xor_sync(0xffffffffu, w, o);
       if (a.step > 1) w &= range;
       reinterpret_cast<uint32_t*>(x_words + xs * 128 + r)[qtr] = w;
-      mbar_arrive(bar_x(xs));
+      __syncwarp();                                   // the warp's words, then its one arrival
+      if (lane == 0) mbar_arrive(bar_x(xs));
       if (!warp_wait(bar_x(xs), (t >> 1) & 1, wc)) break;
       const uint4 mine = x_words[xs * 128 + r];            // this row's four words
       const uint32_t* mw = &mine.x;
@@ -775,8 +775,7 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
       }
       // append.  When every row of the warp keeps all 32 keys of its word (the
       // dense case), every row stores the same 32 values: one shuffle and one
-      // coalesced store per row.  Otherwise stage (word, list position) and
-      // store each row's set bits.
+      // coalesced store per row.
       const int key = key0 + lane;
       const int pos = row_elem + off + before;
       const bool dense = __all_sync(0xffffffffu, w == 0xffffffffu);
@@ -785,13 +784,11 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) hl[__shfl_sync(0xffffffffu, pos, j)] = key;
       }
-      // rows with keys still to store
-      const uint32_t need = __ballot_sync(0xffffffffu, !dense && w != 0u);
-      // few keys per row (every word of the warp at most 8 bits): each thread
-      // stores its own row's keys, one per step, instead of a warp-wide store
-      // per row
-      const bool sparse = need != 0u && __reduce_max_sync(0xffffffffu, __popc(w)) <= 8;
-      if (sparse) {
+      const int most = dense ? 0 : __reduce_max_sync(0xffffffffu, __popc(w));
+      if (most > 0 && most <= 8) {
+        // few keys per row (every word of the warp at most 8 bits): each
+        // thread stores its own row's keys, one per step, instead of a
+        // warp-wide store per row
         uint32_t rem = w;
         int k = 0;
         while (__any_sync(0xffffffffu, rem != 0u)) {
@@ -800,19 +797,16 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
             rem &= rem - 1u;
           }
         }
-      } else if (need) {
-        my_stage[lane] = make_uint4(w, static_cast<uint32_t>(pos), 0u, 0u);
-        __syncwarp();
-        for (uint32_t rows = need; rows; rows &= rows - 1u) {
-          const int j = __ffs(rows) - 1;
-          const uint4 v = my_stage[j];
-          if (v.x == 0xffffffffu) {
-            head_lists[static_cast<int>(v.y) + lane] = key;
-          } else if ((v.x >> lane) & 1u) {
-            head_lists[static_cast<int>(v.y) + __popc(v.x & lt)] = key;
-          }
+      } else if (most > 8) {
+        // otherwise row by row, lane l storing key l at its rank in the row's
+        // word; the rows' words and positions come by shuffle, eight rows in
+        // flight at a time
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) {
+          const uint32_t wj = __shfl_sync(0xffffffffu, w, j);
+          const int pj = __shfl_sync(0xffffffffu, pos, j);
+          if ((wj >> lane) & 1u) head_lists[pj + __popc(wj & lt)] = key;
         }
-        __syncwarp();
       }
       off += total;
     }

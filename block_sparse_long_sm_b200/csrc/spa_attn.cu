@@ -29,12 +29,14 @@ SPA_API spa_status sparse_prefill_attn(const spa_params* p, const void* q, const
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return SPA_ERR_INVALID;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const long long BH = (long long)B * Hq, BKV = (long long)B * Hkv;
-  CUtensorMap tq, tk, tkg, tv, tvg;
+  CUtensorMap tq, tk, tkg, tv, tvg, tk16, tv16;
   if (!map_2d(&tq, kBF16, 2, q, 128, BH * L, 64, 128, kSW128) ||
       !map_2d(&tk, kBF16, 2, k, 128, BKV * L, 64, 128, kSW128) ||
       !map_2d(&tkg, kBF16, 2, k, 128, BKV * L, 64, 1, kSW128) ||
       !map_2d(&tv, kBF16, 2, v, 128, BKV * L, 64, 128, kSW128) ||
-      !map_2d(&tvg, kBF16, 2, v, 128, BKV * L, 64, 1, kSW128))
+      !map_2d(&tvg, kBF16, 2, v, 128, BKV * L, 64, 1, kSW128) ||
+      !map_2d(&tk16, kBF16, 2, k, 128, BKV * L, 64, 16, kSW128) ||
+      !map_2d(&tv16, kBF16, 2, v, 128, BKV * L, 64, 16, kSW128))
     return SPA_ERR_CUDA;
   AttnArgs aa{};
   aa.B = B; aa.Hq = Hq; aa.Hkv = Hkv; aa.L = L; aa.nqb = lo.nqb; aa.group = lo.group;
@@ -62,7 +64,7 @@ SPA_API spa_status sparse_prefill_attn(const spa_params* p, const void* q, const
   if (lo.paired) {
     if (set_smem(sparse_attn_pair_kernel, kPairSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
     sparse_attn_pair_kernel<<<(unsigned)(lo.nb / 2), kPairThreads, kPairSmemBytes, stream>>>(
-        tq, tk, tkg, tv, tvg, aa);
+        tq, tk, tkg, tv, tvg, tk16, tv16, aa);
   } else {
     if (set_smem(sparse_attn_kernel, kAttnSmemBytes) != cudaSuccess) return SPA_ERR_CUDA;
     sparse_attn_kernel<<<(unsigned)lo.nb, kAttnThreads, kAttnSmemBytes, stream>>>(tq, tk, tkg,
