@@ -7,12 +7,14 @@
 //
 // One CTA = (b, kv head, query block, head pair (2p, 2p+1)).  Its key tiles:
 //   sink tiles       keys [0, sink_end), contiguous;
-//   dense tiles      candidate tiles (128 aligned keys) in which the two
-//                    heads keep at least kTileDenseMin keys together: loaded
+//   dense tiles      candidate tiles (128 aligned keys) of which either
+//                    head keeps at least tile_dense_min keys (64 of keys
+//                    selected one by one, all 128 of key blocks): loaded
 //                    contiguously, the keys a head did not keep masked out of
 //                    its softmax;
 //   gathered tiles   the kept keys of the sparser candidate tiles, 128 at a
-//                    time (the last one padded), copied row by row;
+//                    time (the last one padded), copied row by row, or 16
+//                    consecutive keys at once;
 //   local tiles      keys [ls, row0 + 128), contiguous; the last one is the
 //                    causally masked diagonal.
 // They are loaded in the order sink, dense, local before the diagonal,

@@ -39,11 +39,13 @@ __host__ __device__ __forceinline__ long long tmask_prefix(long long n, int c) {
 // Tile bitmaps.  Beside the masks the plan writes, per (b, h, query block),
 // three bitmaps over the block's candidate tiles (bit t of word t / 32 <=>
 // candidate tile kt0 + t), each tmask_bit_words(nqb, c) words long:
-// non-empty (some key kept), dense (at least kTileDenseMin keys kept) and
-// full (all 128 keys kept).  The paired attention kernel walks its tiles from
-// them: a tile a head pair keeps densely is loaded whole, the keys of the
-// others are gathered.
-constexpr int kTileDenseMin = 64;
+// non-empty (some key kept), dense (at least tile_dense_min(unit) keys kept)
+// and full (all 128 keys kept).  The paired attention kernel walks its tiles
+// from them: a tile a head pair keeps densely is loaded whole, the keys of
+// the others are gathered.  Keys selected one by one (unit 1) gather row by
+// row, so a tile half kept is cheaper loaded whole; key blocks of 16 or more
+// keys (SALE) gather as whole boxes, so only a full tile is loaded whole.
+__host__ __device__ __forceinline__ int tile_dense_min(int unit) { return unit > 1 ? 128 : 64; }
 __host__ __device__ __forceinline__ int tmask_bit_words(int nqb, int c) {
   return (tmask_tiles(nqb - 1, c) + 31) / 32;
 }

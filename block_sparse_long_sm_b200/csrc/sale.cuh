@@ -87,20 +87,22 @@ __global__ void __launch_bounds__(128) quant_kernel(const QuantArgs a) {
 // ---------------------------------------------------------------------------
 // fused sink-local statistics + block scan
 // ---------------------------------------------------------------------------
-// One CTA = (b, kv head, query block, up to four q heads of that kv head's
-// group): the q heads share every int8 K tile, so each 64-key tile fetched
-// from L2 feeds up to four MMAs (M = 128 rows, N = 64, K = 128 in four
-// K = 32 steps).  TMEM: two accumulator sets x four heads x 64 columns.  The
-// epilogue (warps 2-9) gives each thread one row of two heads, all 64
-// columns of every tile, so the sink-local statistics need no cross-thread
-// merge.  Candidate tiles are read from TMEM as packed 16-bit pairs (the dots
-// fit: |dot| <= 7*7*128) and reduced with max.s16x2.
+// One CTA = (b, kv head, query block, up to two q heads of that kv head's
+// group): the q heads share every int8 K tile, so each 128-key tile fetched
+// from L2 feeds two MMAs (M = 128 rows, N = 128 keys, K = 128 in four K = 32
+// steps; few, large MMAs, since the issue of an int8 MMA of N = 64 costs
+// about what it computes).  TMEM: two accumulator sets x two heads x 128
+// columns.  The epilogue (warps 2-9) gives each thread one row of one head,
+// all 128 columns of every tile, so the sink-local statistics need no
+// cross-thread merge.  Candidate tiles are read from TMEM as packed 16-bit
+// pairs (the dots fit: |dot| <= 7*7*128) and reduced with max.s16x2; the
+// accumulator set is released as soon as it is in registers.
 constexpr int kSaleThreads = 320;            // warp 0 TMA, warp 1 MMA, warps 2-9 epilogue
-constexpr int kSaleStages = 8;
-constexpr int kSaleKeys = 64;                // keys per K tile
-constexpr int kSaleHeads = 4;                // q heads per CTA
-constexpr int kSaleBufs = 2;                 // accumulator sets in TMEM (kSaleBufs * kSaleHeads * 64 <= 512)
-static_assert(kSaleBufs * kSaleHeads * 64 <= 512, "more TMEM columns than a CTA has");
+constexpr int kSaleStages = 6;
+constexpr int kSaleKeys = 128;               // keys per K tile
+constexpr int kSaleHeads = 2;                // q heads per CTA
+constexpr int kSaleBufs = 2;                 // accumulator sets in TMEM
+static_assert(kSaleBufs * kSaleHeads * kSaleKeys <= 512, "more TMEM columns than a CTA has");
 constexpr uint32_t kQ8Bytes = 128u * 128u;   // 128 rows x 128 int8
 constexpr uint32_t kK8Bytes = kSaleKeys * 128u;
 constexpr int kMaxGroupWords = 512;          // candidate 16-key groups / 32 (L <= 262144)
@@ -108,7 +110,7 @@ constexpr int kMaxScales = 16384;            // key blocks per head (L / bk <= 1
 constexpr uint32_t kSaleSmemBytes = 1024u + kSaleHeads * kQ8Bytes + kSaleStages * kK8Bytes +
                                     1024u + kSaleHeads * kMaxGroupWords * 4u + kMaxScales * 4u;
 static_assert(kSaleSmemBytes <= 232448u, "more shared memory than a CTA may use");
-constexpr uint32_t kIdescI8N64 = make_idesc(2, 1, 128, 64, 0, 0);
+constexpr uint32_t kIdescI8N128 = make_idesc(2, 1, 128, 128, 0, 0);
 
 struct SaleArgs {
   int B, Hq, Hkv, L, nqb, group;
@@ -233,9 +235,9 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
         for (int j = 0; j < nh; ++j) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            mma_i8_ss(tmem + 64u * (bb * kSaleHeads + j),
+            mma_i8_ss(tmem + static_cast<uint32_t>(kSaleKeys) * (bb * kSaleHeads + j),
                       smem_desc_sw128(s_q + j * kQ8Bytes + kk * 32u, 16),
-                      smem_desc_sw128(s_k(st) + kk * 32u, 16), kIdescI8N64, kk > 0 ? 1u : 0u);
+                      smem_desc_sw128(s_k(st) + kk * 32u, 16), kIdescI8N128, kk > 0 ? 1u : 0u);
           }
         }
         mma_commit(bar_afull(bb));
@@ -247,108 +249,98 @@ sale_scan_kernel(const __grid_constant__ CUtensorMap tm_q8,
     __syncwarp();
   } else {
     const int quad = warp & 3;               // TMEM lane quadrant
-    const int hsel = (warp - 2) >> 2;        // heads hsel and hsel + 2
+    const int hsel = (warp - 2) >> 2;        // head h0 + hsel
+    const bool head_valid = hsel < nh;       // warp-uniform
     const int r = quad * 32 + lane;
     const int row = row0 + r;
     const bool row_valid = row < a.L;
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    float cq[2], m[2], l[2], thr[2];
-#pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      const int j = hsel + 2 * u;
-      cq[u] = j < nh ? a.sq[((long long)b * a.Hq + h0 + j) * a.nqb + qb] : 0.f;
-      m[u] = -INFINITY;
-      l[u] = 0.f;
-      thr[u] = INFINITY;
-    }
+    const float cq = head_valid ? a.sq[((long long)b * a.Hq + h0 + hsel) * a.nqb + qb] : 0.f;
+    float m = -INFINITY, l = 0.f, thr = INFINITY;
     for (int t = 0; t < T; ++t) {
       const int bb = t % kSaleBufs;
       if (!warp_wait(bar_afull(bb), (t / kSaleBufs) & 1, wc)) break;
       tc_fence_after();
       const int key0 = tile_key0(t);
-      if (t < n_stat_t) {
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int j = hsel + 2 * u;
-          if (j >= nh) continue;                       // warp-uniform
-          const uint32_t taddr = tmem + lane_off + 64u * (bb * kSaleHeads + j);
+      const uint32_t taddr = tmem + lane_off + static_cast<uint32_t>(kSaleKeys) * (bb * kSaleHeads + hsel);
+      bool released = false;
+      if (head_valid && t < n_stat_t) {
+        // S~ over the causal sink-local keys of this row, 64 columns at a time
+        int limit = (t < n_sink_t) ? sink_end - key0 : min(le - key0, row - key0 + 1);
+        limit = max(0, min(limit, kSaleKeys));
+#pragma unroll 1
+        for (int half = 0; half < 2; ++half) {
           uint32_t sr[2][32];
-          tmem_ld32(taddr, sr[0]);
-          tmem_ld32(taddr + 32u, sr[1]);
+          tmem_ld32(taddr + 64u * half, sr[0]);
+          tmem_ld32(taddr + 64u * half + 32u, sr[1]);
           tmem_ld_wait();
-          // S~ over the causal sink-local keys of this row
-          int limit = (t < n_sink_t) ? sink_end - key0 : min(le - key0, row - key0 + 1);
-          limit = max(0, min(limit, kSaleKeys));
           float tm = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const int col = c * 32 + e;
+              const int col = 64 * half + c * 32 + e;
               const float v = col < limit
                                   ? static_cast<float>(static_cast<int>(sr[c][e])) *
-                                        (cq[u] * kscale[min(key0 + col, a.L - 1) >> a.bk_log2])
+                                        (cq * kscale[min(key0 + col, a.L - 1) >> a.bk_log2])
                                   : -INFINITY;
               sr[c][e] = __float_as_uint(v);
               tm = fmaxf(tm, v);
             }
           }
           if (tm > -INFINITY) {
-            const float mn = fmaxf(m[u], tm);
+            const float mn = fmaxf(m, tm);
             float acc = 0.f;
 #pragma unroll
             for (int c = 0; c < 2; ++c)
 #pragma unroll
               for (int e = 0; e < 32; ++e) acc += __expf(__uint_as_float(sr[c][e]) - mn);
-            l[u] = l[u] * __expf(m[u] - mn) + acc;
-            m[u] = mn;
+            l = l * __expf(m - mn) + acc;
+            m = mn;
           }
-          if (t == n_stat_t - 1)
-            thr[u] = row_valid ? m[u] + logf(a.tau_h[h0 + hsel + 2 * u] * l[u])   // t_i = em + ln(tau el)
-                               : INFINITY;
         }
-      } else {
-        // both heads' 64 columns as packed 16-bit pairs, one wait for the two
-        // loads; the four 16-key groups' K scales are read meanwhile
+        if (t == n_stat_t - 1)
+          thr = row_valid ? m + logf(a.tau_h[h0 + hsel] * l) : INFINITY;   // t_i = em + ln(tau el)
+      } else if (head_valid) {
+        // the 128 columns as packed 16-bit pairs, one wait for the two loads;
+        // the eight 16-key groups' K scales are read meanwhile
         uint32_t pk[2][32];
+        tmem_ld32_pack16(taddr, pk[0]);
+        tmem_ld32_pack16(taddr + 64u, pk[1]);
+        float ksg[8];
 #pragma unroll
-        for (int u = 0; u < 2; ++u)
-          if (hsel + 2 * u < nh) tmem_ld32_pack16(tmem + lane_off + 64u * (bb * kSaleHeads + hsel + 2 * u), pk[u]);
-        float ksg[4];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) ksg[g] = kscale[min(key0 + 16 * g, cand_hi - 1) >> a.bk_log2];
+        for (int g = 0; g < 8; ++g) ksg[g] = kscale[min(key0 + 16 * g, cand_hi - 1) >> a.bk_log2];
         tmem_ld_wait();
-        uint32_t gbits = 0;                            // bit 4u + g: head hsel + 2u, group g
+        // the dots are in registers: the set is free for tile t + kSaleBufs
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_afree(bb));
+        released = true;
+        uint32_t gbits = 0;                            // bit g: 16-key group g of the tile
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          if (hsel + 2 * u >= nh) continue;            // warp-uniform
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {                // 16 keys = 8 packed registers
-            const uint32_t* q = pk[u] + 8 * g;
-            const uint32_t m01 = max_s16x2(max_s16x2(q[0], q[1]), max_s16x2(q[2], q[3]));
-            const uint32_t m23 = max_s16x2(max_s16x2(q[4], q[5]), max_s16x2(q[6], q[7]));
-            const uint32_t mm = max_s16x2(m01, m23);
-            const int mx = max(static_cast<int>(static_cast<int16_t>(mm & 0xffffu)),
-                               static_cast<int>(mm) >> 16);
-            if (key0 + 16 * g < cand_hi && static_cast<float>(mx) * (cq[u] * ksg[g]) >= thr[u])
-              gbits |= 1u << (4 * u + g);
-          }
+        for (int g = 0; g < 8; ++g) {                  // 16 keys = 8 packed registers
+          const uint32_t* q = pk[g >> 2] + 8 * (g & 3);
+          const uint32_t m01 = max_s16x2(max_s16x2(q[0], q[1]), max_s16x2(q[2], q[3]));
+          const uint32_t m23 = max_s16x2(max_s16x2(q[4], q[5]), max_s16x2(q[6], q[7]));
+          const uint32_t mm = max_s16x2(m01, m23);
+          const int mx = max(static_cast<int>(static_cast<int16_t>(mm & 0xffffu)),
+                             static_cast<int>(mm) >> 16);
+          if (key0 + 16 * g < cand_hi && static_cast<float>(mx) * (cq * ksg[g]) >= thr)
+            gbits |= 1u << g;
         }
-        // one warp reduction and at most two shared atomics per tile for both heads
+        // one warp reduction and at most one shared atomic per tile
         gbits = __reduce_or_sync(0xffffffffu, gbits);
         if (lane == 0 && gbits) {
-          const int g0 = (key0 - cand_lo) / 16;        // multiple of 4: one word holds 4 bits
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const uint32_t bits = (gbits >> (4 * u)) & 0xfu;
-            if (bits) atomicOr(&gflags[(hsel + 2 * u) * kMaxGroupWords + (g0 >> 5)], bits << (g0 & 31));
-          }
+          const int g0 = (key0 - cand_lo) / 16;        // multiple of 8: one word holds the 8 bits
+          atomicOr(&gflags[hsel * kMaxGroupWords + (g0 >> 5)], gbits << (g0 & 31));
         }
       }
-      // the buffer is free once every epilogue warp has read it: one arrival per warp
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar_afree(bb));
+      if (!released) {
+        // the set is free once every epilogue warp has read it: one arrival per warp
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_afree(bb));
+      }
     }
   }
   tc_fence_before();

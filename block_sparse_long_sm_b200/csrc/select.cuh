@@ -547,10 +547,11 @@ stripe_scan_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 // count before its word, and the first four warps store each row's four
 // words as its tile mask.  Stores, by density of the warp's 32 words: all
 // keys kept -- one shuffle and one coalesced store of the same 32 values per
-// row; at most 8 keys in every word -- each thread stores its own row's keys;
-// in between -- row by row, the row's word and list position shuffled to the
-// warp, one coalesced store of its kept keys.  CTAs are numbered heaviest first (last M
-// tile first), so the block scheduler fills the GPU longest-job-first.
+// row; few keys in every word -- each thread stores its own row's keys;
+// otherwise row by row over the rows with keys, the row's word and list
+// position shuffled to the warp, one coalesced store of its kept keys.  CTAs
+// are numbered heaviest first (last M tile first), so the block scheduler
+// fills the GPU longest-job-first.
 constexpr int kSelEpiWarps = 16;
 constexpr int kSelThreads = 32 * (2 + kSelEpiWarps);
 constexpr int kSelStages = 4;
@@ -764,7 +765,7 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
         row_tmask[t] = mine;
         const uint32_t bit = 1u << (t & 31);
         if (total > 0) occ_acc |= bit;
-        if (total >= kTileDenseMin) den_acc |= bit;
+        if (total >= tile_dense_min(1)) den_acc |= bit;
         if (total == 128) full_acc |= bit;
         if ((t & 31) == 31 || t == n_ct - 1) {
           row_bits[t >> 5] = occ_acc;
@@ -784,11 +785,15 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) hl[__shfl_sync(0xffffffffu, pos, j)] = key;
       }
+      // Otherwise either each thread stores its own row's keys, one per step
+      // (as many steps as the fullest row has keys, each store scattered over
+      // the rows), when no row has more than 8 keys, or no more than 16 and
+      // at most half as many as there are rows with keys; or row by row, the
+      // row's word and list position shuffled to the warp and its kept keys
+      // stored coalesced (as many steps as rows with keys, two in flight).
       const int most = dense ? 0 : __reduce_max_sync(0xffffffffu, __popc(w));
-      if (most > 0 && most <= 8) {
-        // few keys per row (every word of the warp at most 8 bits): each
-        // thread stores its own row's keys, one per step, instead of a
-        // warp-wide store per row
+      const uint32_t need = __ballot_sync(0xffffffffu, w != 0u);
+      if (most > 0 && (most <= 8 || (most <= 16 && 2 * most <= __popc(need)))) {
         uint32_t rem = w;
         int k = 0;
         while (__any_sync(0xffffffffu, rem != 0u)) {
@@ -797,15 +802,25 @@ stripe_select_kernel(const __grid_constant__ CUtensorMap tm_qbar,
             rem &= rem - 1u;
           }
         }
-      } else if (most > 8) {
-        // otherwise row by row, lane l storing key l at its rank in the row's
-        // word; the rows' words and positions come by shuffle, eight rows in
-        // flight at a time
+      } else if (most > 0 && need == 0xffffffffu) {
 #pragma unroll 8
         for (int j = 0; j < 32; ++j) {
           const uint32_t wj = __shfl_sync(0xffffffffu, w, j);
           const int pj = __shfl_sync(0xffffffffu, pos, j);
           if ((wj >> lane) & 1u) head_lists[pj + __popc(wj & lt)] = key;
+        }
+      } else if (most > 0) {
+        for (uint32_t rest = need; rest;) {
+          const int j0 = __ffs(rest) - 1;
+          rest &= rest - 1u;
+          const int j1 = rest ? __ffs(rest) - 1 : -1;
+          rest &= rest - 1u;
+          const uint32_t w0 = __shfl_sync(0xffffffffu, w, j0);
+          const int p0 = __shfl_sync(0xffffffffu, pos, j0);
+          const uint32_t w1 = __shfl_sync(0xffffffffu, w, j1 & 31);
+          const int p1 = __shfl_sync(0xffffffffu, pos, j1 & 31);
+          if ((w0 >> lane) & 1u) head_lists[p0 + __popc(w0 & lt)] = key;
+          if (j1 >= 0 && ((w1 >> lane) & 1u)) head_lists[p1 + __popc(w1 & lt)] = key;
         }
       }
       off += total;
@@ -985,7 +1000,7 @@ __global__ void __launch_bounds__(128) tile_mask_kernel(const TileMaskArgs a) {
     }
     const int c = __popc(w4[0]) + __popc(w4[1]) + __popc(w4[2]) + __popc(w4[3]);
     const uint32_t occ = __ballot_sync(0xffffffffu, c > 0);
-    const uint32_t den = __ballot_sync(0xffffffffu, c >= kTileDenseMin);
+    const uint32_t den = __ballot_sync(0xffffffffu, c >= tile_dense_min(a.unit));
     const uint32_t full = __ballot_sync(0xffffffffu, c == 128);
     if (lane == 0) {
       bits[t0 >> 5] = occ;

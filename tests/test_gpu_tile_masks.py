@@ -3,16 +3,19 @@
 For every query block the plan writes, beside the ascending list of kept
 candidate keys, one 128-bit mask per candidate tile (keys 128 kt .. 128 kt +
 127 for sink / 128 <= kt < ls / 128), which the paired attention kernel cuts
-its tiles from, and three bitmaps over the candidate tiles (some key kept,
-at least 64 kept, all 128 kept).  All are read back from the workspace here:
-the masks must spell out the list key for key and the bitmaps must agree
-with the masks' counts, on fused selection (steps 1 and 2), the
+its tiles from, and three bitmaps over the candidate tiles (some key kept;
+at least 64 kept, or all 128 for SALE's key blocks; all 128 kept).  All are
+read back from the workspace here: the masks must spell out the list key
+for key and the bitmaps must agree with the masks' counts, on fused
+selection (steps 1 and 2), the
 bitmask path (step 3), SALE key blocks of every size, a sink that is not a
 multiple of 128, ragged lengths, one and two heads per kv head.
 """
 
 import numpy as np
 import pytest
+
+import block_sparse_long_sm_b200 as spa
 
 from workloads import C0_TINY, generate
 
@@ -39,6 +42,9 @@ def _check(run: Run):
     bstart = ws.size - al(bbytes)
     bitmaps = ws[bstart:bstart + bbytes].view(np.uint32).reshape(run.B * run.Hq, nqb, 3, W)
     kt0 = p.sink // 128
+    # "dense": half the tile for keys selected one by one, the whole tile for
+    # SALE's key blocks (which the attention gathers as whole boxes)
+    dense_min = 128 if p.mode == spa.SPA_MODE_SALE else 64
     checked = 0
     for b in range(run.B):
         for h in range(run.Hq):
@@ -49,12 +55,12 @@ def _check(run: Run):
                 keys = (np.nonzero(bits.reshape(-1))[0] + 128 * kt0).astype(np.int64)
                 want = run.selected_keys(b, h, qb)
                 assert np.array_equal(keys, want), (b, h, qb, keys[:8], want[:8])
-                # the block's bitmaps: non-empty, at least 64 kept, all 128 kept
+                # the block's bitmaps: non-empty, dense, all 128 kept
                 per_tile = bits.sum(axis=1)
                 flags = np.unpackbits(bitmaps[b * run.Hq + h, qb].view(np.uint8),
                                       bitorder="little").reshape(3, -1)[:, :n]
                 assert np.array_equal(flags[0], per_tile > 0), (b, h, qb)
-                assert np.array_equal(flags[1], per_tile >= 64), (b, h, qb)
+                assert np.array_equal(flags[1], per_tile >= dense_min), (b, h, qb)
                 assert np.array_equal(flags[2], per_tile == 128), (b, h, qb)
                 checked += 1
     return checked
