@@ -765,15 +765,21 @@ sparse_attn_pair_kernel(const __grid_constant__ CUtensorMap tm_q,
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + s_col + 32u * c, sr[c]);
       tmem_ld_wait();
+      // the column bound folded into the membership words, so that a column
+      // costs one bit test and one select
       const bool masked = (limit < 128) || ((tw[0] & tw[1] & tw[2] & tw[3]) != 0xffffffffu);
       if (masked) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < 4; ++c) {
+          const int n = limit - 32 * c;
+          const uint32_t keep = tw[c] & (n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : ((1u << n) - 1u)));
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const bool v = (c * 32 + e < limit) && ((tw[c] >> e) & 1u);
-            if (!v) sr[c][e] = __float_as_uint(-INFINITY);
+            // all ones when column e is kept: bit e moved to the sign, then spread
+            const uint32_t k = static_cast<uint32_t>(static_cast<int32_t>(keep << (31 - e)) >> 31);
+            sr[c][e] = (sr[c][e] & k) | (0xff800000u & ~k);
           }
+        }
       }
       float mxv[8];
 #pragma unroll
