@@ -59,7 +59,7 @@ def test_c1_llama_32k_sparse_theta():
     compare_outputs(run, inp, rows)
 
 
-@pytest.mark.parametrize("theta", [5.0, 3.0])
+@pytest.mark.parametrize("theta", [5.0, 3.0, 7.0])
 def test_c2_llama_128k_sampled(theta):
     w = C2_LLAMA_128K
     inp = generate(w)
