@@ -10,7 +10,7 @@
 //       K is smoothed first; an all-zero block gets scale 1.
 //   sale_scan_kernel
 //       per query block on the int8 tensor cores (tcgen05 kind::i8, M = 128,
-//       N = 256): first the sink-local tiles give em_i, el_i and the row
+//       N = 128): first the sink-local tiles give em_i, el_i and the row
 //       threshold t_i = em_i + ln(tau * el_i) (Eq. (4) as corrected); then
 //       every candidate tile: a key block is kept when some valid row's
 //       largest estimated score in it reaches t_i.  The integer dot products
