@@ -160,7 +160,9 @@ SPA_API spa_status sparse_prefill_plan(const spa_params* p, const void* q, const
                                cudaStream_t stream);
 
 /* Attention over sink + selected + local keys (all causal keys in DENSE
- * mode).  Reads q, k, v and the plan's lists; writes o and, when lse is not
+ * mode).  Reads q, k, v and the plan's selection in the workspace (with
+ * Hq / Hkv even, the per-tile keep masks the plan writes in its scratch
+ * beside the lists; otherwise the lists); writes o and, when lse is not
  * NULL, lse.  Records device-side errors in the workspace error word. */
 SPA_API spa_status sparse_prefill_attn(const spa_params* p, const void* q, const void* k,
                                const void* v, void* workspace, size_t workspace_bytes,
